@@ -1,0 +1,115 @@
+// Internal declarations shared by the kernels and the host entry points of
+// libqsa.so (B200, sm_100a).  Nothing here is part of the public ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/qsa.h"
+
+namespace qsa {
+
+// ---- fixed method parameters (validated on the host) ----
+constexpr int kBlock = 4;        // tokens per micro-block
+constexpr int kTopK = 512;       // blocks kept per query
+constexpr int kIdxHeads = 4;     // indexer heads
+constexpr int kIdxDim = 64;      // indexer head dim
+constexpr int kHeadDim = 128;    // main attention head dim
+constexpr int kMaxGroup = 16;    // query heads per KV head handled by one attention CTA
+
+// ---- top-k radix select: 32-bit orderable keys, digits of 12 + 12 + 8 bits ----
+constexpr int kBins1 = 4096;
+constexpr int kBins2 = 4096;
+constexpr int kBins3 = 256;
+
+enum SelectMode : int {
+    kSelUndecided = 0,  // more digits needed
+    kSelAll = 1,        // n_c <= top_k: every candidate
+    kSelPrefix = 2,     // keys whose top `nbits` exceed or equal `prefix`
+    kSelTies = 3,       // keys above `prefix` (full 32 bits) and the first `need` equal ones
+};
+
+// Per-query control block of the decode select, zeroed before every select.
+struct TopkCtrl {
+    unsigned hist1[kBins1];
+    unsigned hist2[kBins2];
+    unsigned hist3[kBins3];
+    unsigned done[4];      // CTA completion counters of the passes
+    unsigned nsel;         // entries appended to the unordered list
+    unsigned prefix;       // resolved high bits of the threshold key
+    int nbits;             // how many high bits are resolved
+    int need;              // entries still to take from keys equal to `prefix`
+    int mode;              // SelectMode
+    int n_cand;            // n_c of the query (after the max_blocks cut)
+    unsigned pad[6];
+};
+static_assert(sizeof(TopkCtrl) % 64 == 0, "TopkCtrl keeps 64-byte alignment");
+
+// fp32 -> unsigned key with the same order (larger float -> larger key); -0 maps to +0.
+__device__ __forceinline__ unsigned orderable_key(float f)
+{
+    unsigned u = __float_as_uint(f);
+    if (u == 0x80000000u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ void set_status(unsigned* status, unsigned bit)
+{
+    if (status) atomicOr(status, bit);
+}
+
+// two bf16 packed in a 32-bit word -> two fp32 (exact)
+__device__ __forceinline__ float bf16lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
+
+// ---- workspace layout ----
+struct WsLayout {
+    size_t status = 0;     // u32 status word (first 256 bytes)
+    size_t ctrl = 0;       // TopkCtrl[n_q] then attention counters u32[n_q * n_kv_heads]
+    size_t ctrl_bytes = 0; // bytes zeroed at the start of each select/attention
+    size_t attn_cnt = 0;   // offset of the attention split counters (inside ctrl)
+    size_t lh3 = 0;        // u32 [n_q][n_chunks][256] per-chunk digit-3 histograms
+    size_t tmp = 0;        // i32 [n_q][top_k] unordered selection
+    size_t scores = 0;     // f32 [n_rows][ld] decode score rows
+    int64_t score_ld = 0;
+    int32_t score_rows = 0;
+    size_t sel = 0;        // i32 [n_q][top_k] + i32 [n_q] when the caller passes none
+    size_t partial = 0;    // f32 split-K partials
+    size_t total = 0;
+    int n_chunks = 0;
+    int chunk = 0;
+    int n_split = 1;
+};
+
+// Chunk of candidate blocks one CTA of the decode scoring/select passes handles.
+int select_chunk(int64_t max_blocks, int32_t n_rows);
+// Split-K factor of the decode attention.
+int attn_splits(int32_t n_q, int32_t n_kv_heads);
+WsLayout plan_workspace(const qsa_dims& d, int32_t n_q, int64_t max_blocks, int32_t mode);
+
+// ---- launchers (return cudaGetLastError()) ----
+cudaError_t launch_pool(const qsa_dims& d, const void* idx_k, void* pooled, const int32_t* len_before,
+                        const int32_t* len_after, int32_t max_new_tokens, unsigned* status,
+                        cudaStream_t st);
+
+// Scores for rows [row0, row0 + n_rows) (query i = row0 + r, optionally via row_list).
+// With ctrl != nullptr also builds the digit-1 histogram and runs the first select analysis.
+cudaError_t launch_score_decode(const qsa_dims& d, const void* q_idx, const float* w, const void* pooled,
+                                const int32_t* q_seq, const int32_t* q_pos, int32_t row0, int32_t n_rows,
+                                int64_t max_blocks, float* scores, int64_t ld, int chunk, TopkCtrl* ctrl,
+                                unsigned* status, cudaStream_t st);
+
+// Radix select over score rows [0, n_rows) (query i = row0 + r).  If `hist_done`
+// the digit-1 histogram was built by the scoring kernel.
+cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, int32_t row0, int32_t n_rows,
+                        int64_t max_blocks, int64_t kv_capacity, int chunk, int n_chunks, TopkCtrl* ctrl, unsigned* lh3,
+                        int32_t* tmp, int32_t* sel_idx, int32_t* sel_cnt, bool hist_done, unsigned* status,
+                        cudaStream_t st);
+
+cudaError_t launch_attention(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,
+                             const int32_t* sel_cnt, int32_t n_q, void* out, int n_split, float* partial,
+                             unsigned* counters, unsigned* status, cudaStream_t st);
+
+}  // namespace qsa

@@ -1,0 +1,178 @@
+"""Thin ctypes binding of libqsa.so (the C ABI in include/qsa.h).
+
+Argument marshalling only: every step runs in the CUDA library.  Tensors are
+torch CUDA tensors (device memory and streams come from PyTorch); their
+data_ptr() values and the current stream's handle are passed straight through.
+There is no CPU fallback: if the library or a GPU is missing, calls raise.
+"""
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libqsa.so")
+
+QSA_OK = 0
+QSA_ERR_INVALID_ARG = -1
+QSA_ERR_WORKSPACE_TOO_SMALL = -2
+QSA_ERR_UNSUPPORTED = -3
+QSA_ERR_CUDA = -4
+
+QSA_DEV_BAD_SEQ = 0x1
+QSA_DEV_BAD_POS = 0x2
+QSA_DEV_BLOCKS_OVER = 0x4
+QSA_DEV_BAD_LEN = 0x8
+QSA_DEV_BAD_SEL = 0x10
+QSA_DEV_TOO_MANY_NEW = 0x20
+
+QSA_MODE_DECODE = 0
+QSA_MODE_PREFILL = 1
+
+EXPORTED = (
+    "qsa_workspace_bytes", "qsa_workspace_init", "qsa_read_device_status", "qsa_status_string",
+    "qsa_pool_block_keys", "qsa_index_scores", "qsa_topk_blocks", "qsa_sparse_attn", "qsa_forward",
+)
+
+
+class QsaError(RuntimeError):
+    def __init__(self, fn, code, msg):
+        super().__init__(f"{fn} failed: {msg} ({code})")
+        self.code = code
+
+
+class qsa_dims(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32), ("n_idx_heads", ctypes.c_int32), ("idx_dim", ctypes.c_int32),
+        ("block_size", ctypes.c_int32), ("top_k", ctypes.c_int32), ("kv_capacity", ctypes.c_int64),
+        ("softmax_scale", ctypes.c_float),
+    ]
+
+
+class qsa_forward_args(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+        ("idx_k", ctypes.c_void_p), ("pooled", ctypes.c_void_p), ("q_idx", ctypes.c_void_p),
+        ("w", ctypes.c_void_p), ("len_before", ctypes.c_void_p), ("len_after", ctypes.c_void_p),
+        ("q_seq", ctypes.c_void_p), ("q_pos", ctypes.c_void_p), ("n_q", ctypes.c_int32),
+        ("max_new_tokens", ctypes.c_int32), ("max_blocks", ctypes.c_int64), ("mode", ctypes.c_int32),
+        ("sel_idx", ctypes.c_void_p), ("sel_cnt", ctypes.c_void_p), ("out", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def load(path=LIB_PATH):
+    """Load libqsa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libqsa.so not built at {path}: run `python -m block_sparse_attention_key_b200.build`")
+    L = ctypes.CDLL(path)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    D = ctypes.POINTER(qsa_dims)
+    L.qsa_workspace_bytes.argtypes = [D, I32, I64, I32]
+    L.qsa_workspace_bytes.restype = SZ
+    L.qsa_workspace_init.argtypes = [P, SZ, P]
+    L.qsa_read_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32), P]
+    L.qsa_status_string.argtypes = [ctypes.c_int]
+    L.qsa_status_string.restype = ctypes.c_char_p
+    L.qsa_pool_block_keys.argtypes = [D, P, P, P, P, I32, P, P]
+    L.qsa_index_scores.argtypes = [D, P, P, P, P, P, I32, I64, P, I64, P, P]
+    L.qsa_topk_blocks.argtypes = [D, P, I64, P, I32, I64, P, P, P, SZ, P]
+    L.qsa_sparse_attn.argtypes = [D, P, P, P, P, P, P, P, I32, P, P, SZ, P]
+    L.qsa_forward.argtypes = [D, ctypes.POINTER(qsa_forward_args), P, SZ, P]
+    for name in EXPORTED:
+        if name not in ("qsa_workspace_bytes", "qsa_status_string"):
+            getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def make_dims(batch, n_q_heads, n_kv_heads, kv_capacity, head_dim=128, n_idx_heads=4, idx_dim=64,
+              block_size=4, top_k=512, softmax_scale=0.0):
+    return qsa_dims(batch, n_q_heads, n_kv_heads, head_dim, n_idx_heads, idx_dim, block_size, top_k,
+                    kv_capacity, softmax_scale)
+
+
+def status_string(code):
+    return load().qsa_status_string(code).decode()
+
+
+def _check(fn, rc):
+    if rc != QSA_OK:
+        raise QsaError(fn, rc, status_string(rc))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("libqsa takes CUDA tensors only (no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+# ---------------------------------------------------------------- entry points (same names as the C ABI)
+
+def qsa_workspace_bytes(dims, n_q, max_blocks, mode):
+    return int(load().qsa_workspace_bytes(ctypes.byref(dims), n_q, max_blocks, mode))
+
+
+def qsa_workspace_init(workspace, stream=None):
+    _check("qsa_workspace_init", load().qsa_workspace_init(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                                           _stream(stream)))
+
+
+def qsa_read_device_status(workspace, stream=None):
+    flags = ctypes.c_uint32(0)
+    _check("qsa_read_device_status", load().qsa_read_device_status(_ptr(workspace), ctypes.byref(flags),
+                                                                   _stream(stream)))
+    return flags.value
+
+
+def qsa_pool_block_keys(dims, idx_k, pooled, len_before, len_after, max_new_tokens, workspace=None, stream=None):
+    _check("qsa_pool_block_keys", load().qsa_pool_block_keys(
+        ctypes.byref(dims), _ptr(idx_k), _ptr(pooled), _ptr(len_before), _ptr(len_after), max_new_tokens,
+        _ptr(workspace), _stream(stream)))
+
+
+def qsa_index_scores(dims, q_idx, w, pooled, q_seq, q_pos, n_q, max_blocks, scores, ld_scores,
+                     workspace=None, stream=None):
+    _check("qsa_index_scores", load().qsa_index_scores(
+        ctypes.byref(dims), _ptr(q_idx), _ptr(w), _ptr(pooled), _ptr(q_seq), _ptr(q_pos), n_q, max_blocks,
+        _ptr(scores), ld_scores, _ptr(workspace), _stream(stream)))
+
+
+def qsa_topk_blocks(dims, scores, ld_scores, q_pos, n_q, max_blocks, sel_idx, sel_cnt, workspace, stream=None):
+    _check("qsa_topk_blocks", load().qsa_topk_blocks(
+        ctypes.byref(dims), _ptr(scores), ld_scores, _ptr(q_pos), n_q, max_blocks, _ptr(sel_idx), _ptr(sel_cnt),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def qsa_sparse_attn(dims, q, k_cache, v_cache, q_seq, q_pos, sel_idx, sel_cnt, n_q, out, workspace, stream=None):
+    _check("qsa_sparse_attn", load().qsa_sparse_attn(
+        ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(q_seq), _ptr(q_pos), _ptr(sel_idx),
+        _ptr(sel_cnt), n_q, _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+
+
+def qsa_forward(dims, *, q, k_cache, v_cache, idx_k, pooled, q_idx, w, len_before, len_after, q_seq, q_pos,
+                n_q, max_new_tokens, max_blocks, mode, out, workspace, sel_idx=None, sel_cnt=None, stream=None):
+    args = qsa_forward_args(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(idx_k), _ptr(pooled), _ptr(q_idx),
+                            _ptr(w), _ptr(len_before), _ptr(len_after), _ptr(q_seq), _ptr(q_pos), n_q,
+                            max_new_tokens, max_blocks, mode, _ptr(sel_idx), _ptr(sel_cnt), _ptr(out))
+    _check("qsa_forward", load().qsa_forward(ctypes.byref(dims), ctypes.byref(args), _ptr(workspace),
+                                             workspace.numel() * workspace.element_size(), _stream(stream)))

@@ -1,0 +1,135 @@
+"""CPU-side checks of the C ABI: the library loads, exports what include/qsa.h
+declares, and rejects bad arguments on the host before launching anything."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def qsa():
+    from block_sparse_attention_key_b200 import build, qsa
+    build.build()
+    qsa.load()
+    return qsa
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "qsa.h")).read()
+    return sorted(set(re.findall(r"^(?:int|size_t|const char\*)\s+(qsa_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_five_layer_calls():
+    names = declared_functions()
+    for n in ["qsa_pool_block_keys", "qsa_index_scores", "qsa_topk_blocks", "qsa_sparse_attn", "qsa_forward"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(qsa):
+    lib = qsa.load()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(qsa.EXPORTED) <= set(declared_functions())
+
+
+def test_binding_names_match_abi(qsa):
+    import block_sparse_attention_key_b200 as pkg
+    for name in declared_functions():
+        if name != "qsa_status_string":
+            assert callable(getattr(pkg, name)), name
+
+
+def test_status_strings(qsa):
+    assert qsa.status_string(0) == "QSA_OK"
+    assert qsa.status_string(-1) == "QSA_ERR_INVALID_ARG"
+    assert qsa.status_string(-2) == "QSA_ERR_WORKSPACE_TOO_SMALL"
+    assert qsa.status_string(-3) == "QSA_ERR_UNSUPPORTED"
+    assert qsa.status_string(-4) == "QSA_ERR_CUDA"
+    assert qsa.status_string(-99) == "QSA_ERR_UNKNOWN"
+
+
+def _dims(qsa, **kw):
+    base = dict(batch=16, n_q_heads=32, n_kv_heads=4, kv_capacity=65536)
+    base.update(kw)
+    return qsa.make_dims(**base)
+
+
+def test_workspace_bytes_rejects_bad_dims(qsa):
+    ok = qsa.qsa_workspace_bytes(_dims(qsa), 16, 16384, qsa.QSA_MODE_DECODE)
+    assert ok > 0
+    bad = [dict(block_size=8), dict(top_k=256), dict(head_dim=64), dict(idx_dim=32), dict(n_idx_heads=2),
+           dict(n_q_heads=30), dict(kv_capacity=65537), dict(batch=0), dict(n_q_heads=64, n_kv_heads=2)]
+    for kw in bad:
+        assert qsa.qsa_workspace_bytes(_dims(qsa, **kw), 16, 16384, 0) == 0, kw
+    assert qsa.qsa_workspace_bytes(_dims(qsa), 16, 16385 + 65536 // 4, 0) == 0   # max_blocks > capacity/4
+    assert qsa.qsa_workspace_bytes(_dims(qsa), -1, 16384, 0) == 0
+    assert qsa.qsa_workspace_bytes(_dims(qsa), 16, 16384, 7) == 0
+
+
+def test_workspace_has_no_query_by_block_term_in_prefill(qsa):
+    """Prefill workspace must not grow like n_q x n_blocks (no mask, no score matrix)."""
+    d = _dims(qsa, batch=1, kv_capacity=1 << 20)
+    nb = (1 << 20) // 4
+    w4 = qsa.qsa_workspace_bytes(d, 4096, nb, qsa.QSA_MODE_PREFILL)
+    w8 = qsa.qsa_workspace_bytes(d, 8192, nb, qsa.QSA_MODE_PREFILL)
+    assert 0 < w4 <= w8
+    assert w8 - w4 < 4096 * nb  # far below one byte per extra (query, block) pair
+    assert w8 < 8192 * nb * 4 // 16
+
+
+def test_decode_workspace_is_small(qsa):
+    d = _dims(qsa, batch=4, kv_capacity=1 << 20)
+    w = qsa.qsa_workspace_bytes(d, 4, (1 << 20) // 4, qsa.QSA_MODE_DECODE)
+    assert 0 < w < 64 << 20
+
+
+def _call(fn, *args):
+    return fn(*args)
+
+
+def test_entry_points_reject_null_and_misaligned_pointers_on_host(qsa):
+    lib = qsa.load()
+    d = ctypes.byref(_dims(qsa))
+    P = None
+    # every call below fails validation before touching CUDA
+    assert lib.qsa_pool_block_keys(d, P, P, P, P, 4, P, P) == qsa.QSA_ERR_INVALID_ARG
+    assert lib.qsa_pool_block_keys(d, 17, 32, 32, 32, 4, P, P) == qsa.QSA_ERR_INVALID_ARG  # misaligned
+    assert lib.qsa_index_scores(d, P, P, P, P, P, 16, 16384, P, 16384, P, P) == qsa.QSA_ERR_INVALID_ARG
+    assert lib.qsa_index_scores(d, 16, 16, 16, 16, 16, 16, 16384, 16, 100, P, P) == qsa.QSA_ERR_INVALID_ARG
+    assert lib.qsa_topk_blocks(d, P, 16384, P, 16, 16384, P, P, P, 0, P) == qsa.QSA_ERR_INVALID_ARG
+    assert lib.qsa_sparse_attn(d, P, P, P, P, P, P, P, 16, P, P, 0, P) == qsa.QSA_ERR_INVALID_ARG
+    args = qsa.qsa_forward_args()
+    args.n_q = 16
+    args.max_blocks = 16384
+    assert lib.qsa_forward(d, ctypes.byref(args), P, 0, P) == qsa.QSA_ERR_INVALID_ARG
+    assert lib.qsa_forward(d, None, 16, 1 << 20, P) == qsa.QSA_ERR_INVALID_ARG
+    assert lib.qsa_workspace_init(P, 0, P) == qsa.QSA_ERR_INVALID_ARG
+    assert lib.qsa_read_device_status(P, None, P) == qsa.QSA_ERR_INVALID_ARG
+
+
+def test_workspace_too_small_is_reported_before_launch(qsa):
+    lib = qsa.load()
+    dims = _dims(qsa)
+    d = ctypes.byref(dims)
+    need = qsa.qsa_workspace_bytes(dims, 16, 16384, 0)
+    fake = 1 << 40  # 16-byte aligned, never dereferenced: the size check fails first
+    rc = lib.qsa_topk_blocks(d, fake, 16384, fake, 16, 16384, fake, fake, fake, need - 1, None)
+    assert rc == qsa.QSA_ERR_WORKSPACE_TOO_SMALL
+    args = qsa.qsa_forward_args(*([fake] * 11), 16, 1, 16384, 0, None, None, fake)
+    assert lib.qsa_forward(d, ctypes.byref(args), fake, need - 1, None) == qsa.QSA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_unsupported_group_size(qsa):
+    lib = qsa.load()
+    d = ctypes.byref(_dims(qsa, n_q_heads=64, n_kv_heads=2))
+    assert lib.qsa_sparse_attn(d, *([16] * 7), 1, 16, 16, 1 << 20, None) == qsa.QSA_ERR_UNSUPPORTED
+
+
+def test_binding_refuses_cpu_tensors(qsa):
+    import torch
+    with pytest.raises(ValueError):
+        qsa._ptr(torch.zeros(4))

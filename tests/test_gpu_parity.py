@@ -1,0 +1,322 @@
+"""GPU parity of each C-ABI step against the CPU oracle, on small seeded inputs
+that span several tiles and ragged tails, plus edge cases."""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+import qsa_synth as syn
+from qsa_synth import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+import gpu_util as gu  # noqa: E402
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    gu.ensure_built()
+    O.lib()
+
+
+def small_workload(name, batch, hq, hkv, cap, steps, mode="decode"):
+    return W.Workload(name, 90 + len(name) % 7, mode, batch, hq, hkv, cap, steps)
+
+
+# ------------------------------------------------------------------ generator twin
+
+def test_device_generator_matches_host_generator():
+    from qsa_synth import device as sdev
+    wl = small_workload("gen", 2, 8, 2, 1024, [W._decode_step(2, 1000, 3)])
+    dw = sdev.DeviceWorkload(wl)
+    for s in range(2):
+        for g in range(2):
+            toks = np.arange(0, 1024, 37)
+            for which, cache in (("k", dw.k_cache), ("v", dw.v_cache)):
+                host = syn.gen_kv_rows(wl.seed, which, s, toks, 2, 128)[:, g, :]
+                dev = gu.to_bits(cache[s, g, toks])
+                np.testing.assert_array_equal(dev, host)
+        np.testing.assert_array_equal(gu.to_bits(dw.idx_k[s]), syn.gen_idx_k(wl.seed, s, 0, 1024, 64))
+    T = dw.step_tensors(0)
+    np.testing.assert_array_equal(gu.to_bits(T["q"]), syn.gen_q(wl.seed, [3, 4], 8, 128))
+    np.testing.assert_array_equal(gu.to_bits(T["q_idx"]), syn.gen_q_idx(wl.seed, [3, 4], 4, 64))
+    np.testing.assert_array_equal(T["w"].cpu().numpy(), syn.gen_w(wl.seed, [3, 4], 4))
+
+
+# ------------------------------------------------------------------ step 1: pooling
+
+def test_pool_bit_exact_and_incremental():
+    import block_sparse_attention_key_b200 as qsa
+    wl = small_workload("pool", 3, 8, 1, 2048, [])
+    from qsa_synth import device as sdev
+    dw = sdev.DeviceWorkload(wl)
+    dims = gu.dims_of(wl)
+    ws = gu.new_workspace(256)
+    i32 = lambda v: torch.tensor(v, dtype=torch.int32, device="cuda")
+    # three sequences appended in two calls with ragged boundaries
+    qsa.qsa_pool_block_keys(dims, dw.idx_k, dw.pooled, i32([0, 0, 0]), i32([101, 6, 2048]), 2048, ws)
+    qsa.qsa_pool_block_keys(dims, dw.idx_k, dw.pooled, i32([101, 6, 2048]), i32([203, 7, 2048]), 102, ws)
+    assert qsa.qsa_read_device_status(ws) == 0
+    for s, n_tok in enumerate([203, 7, 2048]):
+        want = O.pool_blocks(syn.gen_idx_k(wl.seed, s, 0, n_tok, 64))
+        got = gu.to_bits(dw.pooled[s, : n_tok // 4])
+        np.testing.assert_array_equal(got, want)
+        # blocks not yet complete stay untouched (zero)
+        assert (gu.to_bits(dw.pooled[s, n_tok // 4:]) == 0).all()
+
+
+def test_pool_general_bf16_values():
+    """Non-integer keys: fp32 sum then one rounding; equals the fp64 mean rounded once
+    unless the fp32 sum itself was inexact (it is exact for these magnitudes)."""
+    import block_sparse_attention_key_b200 as qsa
+    wl = small_workload("poolg", 1, 8, 1, 4096, [])
+    dims = gu.dims_of(wl)
+    rng = np.random.default_rng(5)
+    vals = rng.normal(size=(1, 4096, 64)).astype(np.float32)
+    bits = torch.tensor(vals).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    idx_k = gu.from_bits(bits)
+    pooled = torch.zeros((1, 1024, 64), dtype=torch.bfloat16, device="cuda")
+    i32 = lambda v: torch.tensor(v, dtype=torch.int32, device="cuda")
+    qsa.qsa_pool_block_keys(dims, idx_k, pooled, i32([0]), i32([4096]), 4096)
+    np.testing.assert_array_equal(gu.to_bits(pooled[0]), O.pool_blocks(bits[0]))
+
+
+# ------------------------------------------------------------------ step 2: scores
+
+def test_index_scores_bit_exact_with_ragged_rows():
+    import block_sparse_attention_key_b200 as qsa
+    positions = [0, 3, 5, 1234, 4093, 4095, 2047, 777]
+    seqs = [0, 1, 2, 0, 1, 2, 1, 0]
+    wl = small_workload("score", 3, 8, 1, 4096, [])
+    from qsa_synth import device as sdev
+    dw = sdev.DeviceWorkload(wl)
+    dims = gu.dims_of(wl)
+    i32 = lambda v: torch.tensor(v, dtype=torch.int32, device="cuda")
+    qsa.qsa_pool_block_keys(dims, dw.idx_k, dw.pooled, i32([0] * 3), i32([4096] * 3), 4096)
+    n = len(positions)
+    qid = list(range(50, 50 + n))
+    q_idx = gu.from_bits(syn.gen_q_idx(wl.seed, qid, 4, 64))
+    w = torch.tensor(syn.gen_w(wl.seed, qid, 4), device="cuda")
+    max_blocks, ld = 1024, 1028
+    scores = torch.full((n, ld), 7.0, device="cuda")
+    ws = gu.new_workspace(256)
+    qsa.qsa_index_scores(dims, q_idx, w, dw.pooled, i32(seqs), i32(positions), n, max_blocks, scores, ld, ws)
+    assert qsa.qsa_read_device_status(ws) == 0
+    got = scores.cpu().numpy()
+    for r, (s, t) in enumerate(zip(seqs, positions)):
+        n_c = (t + 1) // 4
+        pooled = O.pool_blocks(syn.gen_idx_k(wl.seed, s, 0, 4 * n_c, 64))
+        want = O.block_scores(syn.gen_q_idx(wl.seed, [qid[r]], 4, 64)[0], syn.gen_w(wl.seed, [qid[r]], 4)[0], pooled)
+        np.testing.assert_array_equal(got[r, :n_c].astype(np.float64), want)
+        assert np.isneginf(got[r, n_c:max_blocks]).all()
+        assert (got[r, max_blocks:] == 7.0).all()  # padding columns untouched
+
+
+# ------------------------------------------------------------------ step 3: top-k
+
+def _run_topk(score_rows, positions, max_blocks):
+    import block_sparse_attention_key_b200 as qsa
+    wl = small_workload("topk", 1, 8, 1, 4 * max_blocks + 4, [])
+    dims = gu.dims_of(wl)
+    n = len(positions)
+    ld = (max_blocks + 3) // 4 * 4
+    sc = np.full((n, ld), -np.inf, dtype=np.float32)
+    for r, row in enumerate(score_rows):
+        sc[r, : len(row)] = row
+    scores = torch.tensor(sc, device="cuda")
+    q_pos = torch.tensor(positions, dtype=torch.int32, device="cuda")
+    sel_idx = torch.empty((n, 512), dtype=torch.int32, device="cuda")
+    sel_cnt = torch.empty((n,), dtype=torch.int32, device="cuda")
+    ws = gu.new_workspace(qsa.qsa_workspace_bytes(dims, n, max_blocks, 0))
+    qsa.qsa_topk_blocks(dims, scores, ld, q_pos, n, max_blocks, sel_idx, sel_cnt, ws)
+    assert qsa.qsa_read_device_status(ws) == 0
+    return sel_idx.cpu().numpy(), sel_cnt.cpu().numpy()
+
+
+def test_topk_matches_oracle_on_ties_and_ragged_counts():
+    rng = np.random.default_rng(17)
+    n_cs = [0, 1, 511, 512, 513, 700, 5000, 20000, 20000, 20000, 20000, 3]
+    rows = [
+        rng.integers(0, 4, n_cs[0]), rng.integers(0, 4, 1), rng.integers(0, 9, 511), rng.integers(0, 3, 512),
+        rng.integers(0, 3, 513), rng.normal(size=700), rng.integers(0, 50, 5000) * 0.25,
+        np.zeros(20000),                                   # tie storm: lowest 512 indices
+        rng.integers(-5, 5, 20000).astype(np.float64),     # negative scores, ties at the cut
+        np.linspace(0, 1, 20000)[::-1].copy(),             # strictly decreasing: first 512
+        np.where(rng.random(20000) < 0.5, -0.0, 0.0),      # signed zeros compare equal
+        np.array([1.0, 1.0, 1.0]),
+    ]
+    rows = [np.asarray(r, dtype=np.float32) for r in rows]
+    positions = [4 * c for c in n_cs]  # n_c(t) = c exactly (one partial token)
+    sel, cnt = _run_topk(rows, positions, max_blocks=20000)
+    for r, row in enumerate(rows):
+        want = O.select_top_blocks(row.astype(np.float64), 512)
+        assert cnt[r] == len(want), r
+        np.testing.assert_array_equal(sel[r, : cnt[r]], want, err_msg=f"row {r}")
+        assert (sel[r, cnt[r]:] == -1).all()
+
+
+def test_topk_partial_positions_use_complete_blocks_only():
+    rng = np.random.default_rng(2)
+    row = rng.integers(0, 100, 4000).astype(np.float32)
+    # t = 4*1000 + {0,1,2}: n_c = 1000 (the block holding t is not a candidate)
+    sel, cnt = _run_topk([row[:1001]] * 3, [4000, 4001, 4002], max_blocks=1001)
+    want = O.select_top_blocks(row[:1000].astype(np.float64), 512)
+    for r in range(3):
+        np.testing.assert_array_equal(sel[r, : cnt[r]], want)
+
+
+# ------------------------------------------------------------------ step 4: attention
+
+@pytest.mark.parametrize("hq,hkv", [(8, 1), (32, 4), (16, 16), (16, 1), (4, 2)])
+def test_sparse_attn_matches_oracle(hq, hkv):
+    import block_sparse_attention_key_b200 as qsa
+    from qsa_synth import device as sdev
+    rng = np.random.default_rng(hq * 100 + hkv)
+    cap = 8192
+    positions = [8191, 4098, 2050, 3, 0, 6001, 2047, 5]
+    seqs = [0, 1, 0, 1, 0, 1, 1, 0]
+    wl = small_workload(f"attn{hq}_{hkv}", 2, hq, hkv, cap, [W.Step([cap] * 2, [cap] * 2, seqs, positions,
+                                                                    list(range(len(positions))))])
+    dw = sdev.DeviceWorkload(wl)
+    T = dw.step_tensors(0)
+    n = len(positions)
+    sel = np.full((n, 512), -1, dtype=np.int32)
+    cnt = np.zeros(n, dtype=np.int32)
+    for r, t in enumerate(positions):
+        n_c = (t + 1) // 4
+        k = min(512, n_c)
+        chosen = np.sort(rng.choice(n_c, size=k, replace=False)) if k else np.zeros(0, np.int64)
+        sel[r, :k] = chosen
+        cnt[r] = k
+    sel_t = torch.tensor(sel, device="cuda")
+    cnt_t = torch.tensor(cnt, device="cuda")
+    dims = gu.dims_of(wl)
+    ws = gu.new_workspace(qsa.qsa_workspace_bytes(dims, n, 0, 0))
+    out = torch.empty((n, hq, 128), dtype=torch.bfloat16, device="cuda")
+    qsa.qsa_sparse_attn(dims, T["q"], dw.k_cache, dw.v_cache, T["q_seq"], T["q_pos"], sel_t, cnt_t, n, out, ws)
+    assert qsa.qsa_read_device_status(ws) == 0
+    got = gu.bf16_to_f64(out)
+    want = np.zeros_like(got)
+    qbits = gu.to_bits(T["q"])
+    for r, (s, t) in enumerate(zip(seqs, positions)):
+        toks = O.attended_tokens(sel[r, : cnt[r]], t)
+        k = syn.gen_kv_rows(wl.seed, "k", s, toks, hkv, 128)
+        v = syn.gen_kv_rows(wl.seed, "v", s, toks, hkv, 128)
+        want[r] = O.gqa_attention(qbits[r], k, v)
+    gu.compare_outputs(got, want)
+
+
+# ------------------------------------------------------------------ whole layer, edge cases
+
+def _forward_vs_oracle(wl, mode=None):
+    from qsa_synth import device as sdev
+    dw = sdev.DeviceWorkload(wl)
+    wo = O.WorkloadOracle(wl)
+    for step in range(len(wl.steps)):
+        if step == 0:
+            gu.pool_history(dw, 0)
+        out, sel_idx, sel_cnt, flags = gu.run_forward(dw, step, mode)
+        assert flags == 0
+        gu.check_selection_properties(wl, step, sel_idx, sel_cnt)
+        got = gu.bf16_to_f64(out)
+        sel = sel_idx.cpu().numpy()
+        cnt = sel_cnt.cpu().numpy()
+        want = np.zeros_like(got)
+        for r in range(len(wl.steps[step].q_pos)):
+            s_want, o_want = wo.query(step, r)
+            np.testing.assert_array_equal(sel[r, : cnt[r]], s_want, err_msg=f"step {step} row {r}")
+            want[r] = o_want
+        gu.compare_outputs(got, want)
+
+
+def test_forward_decode_short_and_ragged_positions():
+    # positions around empty, one-block, partial-block and the 512-block budget edge
+    pos = [0, 1, 2, 3, 4, 7, 2046, 2047, 2048, 2051, 2052, 2055, 3000, 4095]
+    n = len(pos)
+    wl = W.Workload("edge_decode", 97, "decode", n, 8, 2, 4096,
+                    [W.Step([p for p in pos], [p + 1 for p in pos], list(range(n)), pos, list(range(n)))])
+    _forward_vs_oracle(wl)
+
+
+def test_forward_decode_two_steps_block_completion():
+    # step 1 leaves a 3-token partial block, step 2 completes it (it becomes a candidate)
+    cap = 16384
+    wl = W.Workload("two_steps", 98, "decode", 3, 16, 2, cap,
+                    [W._decode_step(3, cap - 2, 0), W._decode_step(3, cap - 1, 3)])
+    _forward_vs_oracle(wl)
+
+
+@pytest.mark.parametrize("hq,hkv", [(32, 4), (8, 8)])
+def test_forward_prefill_chunk(hq, hkv):
+    # 300 queries of one sequence at ragged positions crossing the 512-block edge
+    wl = W.Workload(f"prefill_small_{hq}", 99, "prefill", 1, hq, hkv, 4096, [W._prefill_step(1900, 300)])
+    _forward_vs_oracle(wl)
+
+
+def test_forward_prefill_mode_decode_shapes_agree():
+    """The same queries through both modes give identical selections."""
+    from qsa_synth import device as sdev
+    wl = W.Workload("modes", 96, "prefill", 1, 32, 4, 8192, [W._prefill_step(6000, 64)])
+    dw = sdev.DeviceWorkload(wl)
+    gu.pool_history(dw, 0)
+    out_p, sel_p, cnt_p, f1 = gu.run_forward(dw, 0, mode=1)
+    out_d, sel_d, cnt_d, f2 = gu.run_forward(dw, 0, mode=0)
+    assert f1 == 0 and f2 == 0
+    assert torch.equal(sel_p, sel_d) and torch.equal(cnt_p, cnt_d)
+    gu.compare_outputs(gu.bf16_to_f64(out_d), gu.bf16_to_f64(out_p))
+
+
+# ------------------------------------------------------------------ device-side errors
+
+def test_bad_positions_and_selections_set_status_without_faulting():
+    import block_sparse_attention_key_b200 as qsa
+    from qsa_synth import device as sdev
+    wl = small_workload("bad", 2, 8, 1, 1024, [W.Step([1024] * 2, [1024] * 2, [0, 5, 1], [100, 10, 5000], [0, 1, 2])])
+    dw = sdev.DeviceWorkload(wl)
+    dims = gu.dims_of(wl)
+    T = dw.step_tensors(0)
+    ws = gu.new_workspace(qsa.qsa_workspace_bytes(dims, 3, 256, 0))
+    out = torch.zeros((3, 8, 128), dtype=torch.bfloat16, device="cuda")
+    sel = torch.full((3, 512), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(3, dtype=torch.int32, device="cuda")
+    qsa.qsa_forward(dims, q=T["q"], k_cache=dw.k_cache, v_cache=dw.v_cache, idx_k=dw.idx_k, pooled=dw.pooled,
+                    q_idx=T["q_idx"], w=T["w"], len_before=T["len_before"], len_after=T["len_after"],
+                    q_seq=T["q_seq"], q_pos=T["q_pos"], n_q=3, max_new_tokens=0, max_blocks=256, mode=0,
+                    out=out, workspace=ws, sel_idx=sel, sel_cnt=cnt)
+    flags = qsa.qsa_read_device_status(ws)
+    assert flags & qsa.qsa.QSA_DEV_BAD_SEQ and flags & qsa.qsa.QSA_DEV_BAD_POS
+    assert qsa.qsa_read_device_status(ws) == 0  # reading clears
+    c = cnt.cpu().numpy()
+    assert c[0] == 25 and c[1] == 0 and c[2] == 0
+    assert (gu.bf16_to_f64(out[1:]) == 0).all()
+    # a selection index outside [0, n_c) is skipped and reported
+    bad_sel = sel.clone()
+    bad_sel[0, 0] = 9999
+    qsa.qsa_sparse_attn(dims, T["q"], dw.k_cache, dw.v_cache, T["q_seq"], T["q_pos"], bad_sel, cnt, 3, out, ws)
+    assert qsa.qsa_read_device_status(ws) & qsa.qsa.QSA_DEV_BAD_SEL
+    torch.cuda.synchronize()
+
+
+def test_forward_allocates_no_device_memory():
+    from qsa_synth import device as sdev
+    wl = W.decode_8k()
+    dw = sdev.DeviceWorkload(wl)
+    gu.pool_history(dw, 0)
+    gu.run_forward(dw, 0)  # warm up: module load, workspace
+    import block_sparse_attention_key_b200 as qsa
+    T = dw.step_tensors(0)
+    dims = gu.dims_of(wl)
+    ws = gu.new_workspace(qsa.qsa_workspace_bytes(dims, 1, 2048, 0))
+    out = torch.empty((1, 8, 128), dtype=torch.bfloat16, device="cuda")
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    qsa.qsa_forward(dims, q=T["q"], k_cache=dw.k_cache, v_cache=dw.v_cache, idx_k=dw.idx_k, pooled=dw.pooled,
+                    q_idx=T["q_idx"], w=T["w"], len_before=T["len_before"], len_after=T["len_after"],
+                    q_seq=T["q_seq"], q_pos=T["q_pos"], n_q=1, max_new_tokens=1, max_blocks=2048, mode=0,
+                    out=out, workspace=ws)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free0 == free1
