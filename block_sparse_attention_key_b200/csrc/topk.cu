@@ -42,7 +42,9 @@ k_topk_pass(const float* __restrict__ scores, int64_t ld, const int32_t* __restr
         nbits = c->nbits;
         need = c->need;
     }
-    const int64_t n_c = candidate_blocks(q_pos[row0 + r], kv_capacity, max_blocks);
+    // the first pass derives the candidates from the position; later passes reuse the
+    // count it recorded (which is 0 for a query the scoring pass rejected)
+    const int64_t n_c = kLevel == 1 ? candidate_blocks(q_pos[row0 + r], kv_capacity, max_blocks) : c->n_cand;
     const int64_t b0 = (int64_t)blockIdx.x * chunk;
     const int64_t b1 = min(b0 + (int64_t)chunk, n_c);
     const float* srow = scores + (int64_t)r * ld;
@@ -96,8 +98,7 @@ k_topk_emit(const float* __restrict__ scores, int64_t ld, const int32_t* __restr
     const int r = blockIdx.y;
     const int i = row0 + r;
     TopkCtrl* c = ctrl + r;
-    const int t = q_pos[i];
-    const int64_t n_c = candidate_blocks(t, kv_capacity, max_blocks);
+    const int64_t n_c = c->n_cand;
     const int mode = c->mode;
     const unsigned prefix = c->prefix;
     const int nbits = c->nbits;
