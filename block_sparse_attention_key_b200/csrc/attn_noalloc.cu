@@ -1,0 +1,110 @@
+// Gathered attention for callers that cannot allocate device memory.
+//
+// qsa_sparse_attn needs a caller workspace for its split-K partials and
+// completion counters.  Some callers have no way to provide one: code running
+// under an allocator that forbids new device allocations (a serving engine that
+// reserved all of HBM for its KV cache up front, a CUDA-graph replay path whose
+// memory plan is frozen), or plain C hosts that only hand over the tensors they
+// already own.  This entry point runs the same attention kernel with its
+// scratch taken from a fixed array compiled into the library instead.
+//
+// The scratch is a file-scope __device__ array of kScratchBytes.  Every GPU that
+// loads this library holds that much memory until the process exits.  On the
+// host the array's name is only a stand-in, not a device address, so the first
+// call on each device (with that device current) looks the address up with
+// cudaGetSymbolAddress and caches it; that first call should therefore come
+// before any stream capture.  All calls share the one array and it keeps the
+// previous call's contents: the completion counters are cleared at the start of
+// every call, and calls whose executions overlap on the GPU (for example on two
+// streams) race on it.  Nothing here calls cudaMalloc, cudaFree or any other
+// allocating routine.
+
+#include <cmath>
+#include <mutex>
+
+#include "qsa_internal.cuh"
+
+namespace qsa {
+
+namespace {
+
+constexpr size_t kScratchBytes = 16u << 20;  // 16 MiB: counters + split partials
+constexpr size_t kCounterAlign = 256;
+constexpr int kMaxDevices = 128;
+
+__device__ __align__(256) unsigned char g_attn_scratch[kScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_attn_scratch on the current device (looked up once per device).
+cudaError_t scratch_address(void** out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_attn_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+bool aligned16(const void* p) { return p != nullptr && ((uintptr_t)p & 15u) == 0; }
+
+int check_args(const qsa_dims* d, int32_t n_q)
+{
+    if (!d || d->batch < 1 || d->n_q_heads < 1 || d->n_kv_heads < 1 || d->n_q_heads % d->n_kv_heads != 0)
+        return QSA_ERR_INVALID_ARG;
+    if (d->block_size != kBlock || d->top_k != kTopK || d->kv_capacity <= 0 || d->kv_capacity % kBlock != 0 ||
+        d->kv_capacity >= (1ll << 31) || !std::isfinite(d->softmax_scale) || n_q < 0)
+        return QSA_ERR_INVALID_ARG;
+    if (d->head_dim != kHeadDim || d->n_idx_heads != kIdxHeads || d->idx_dim != kIdxDim ||
+        d->n_q_heads / d->n_kv_heads > kMaxGroup || n_q > 65535)
+        return QSA_ERR_UNSUPPORTED;
+    return QSA_OK;
+}
+
+}  // namespace
+
+}  // namespace qsa
+
+using namespace qsa;
+
+extern "C" int qsa_sparse_attn_noalloc(const qsa_dims* dims, const void* q, const void* k_cache,
+                                       const void* v_cache, const int32_t* q_seq, const int32_t* q_pos,
+                                       const int32_t* sel_idx, const int32_t* sel_cnt, int32_t n_q, void* out,
+                                       void* stream)
+{
+    // same argument rules as qsa_sparse_attn, minus the workspace
+    const int rc = check_args(dims, n_q);
+    if (rc != QSA_OK) return rc;
+    if (n_q == 0) return QSA_OK;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(q_seq) || !aligned16(q_pos) ||
+        !aligned16(sel_idx) || !aligned16(sel_cnt) || !aligned16(out))
+        return QSA_ERR_INVALID_ARG;
+
+    const int n_split = attn_splits(n_q, dims->n_kv_heads);
+    const size_t counter_bytes = ((size_t)n_q * dims->n_kv_heads * 4 + kCounterAlign - 1) / kCounterAlign *
+                                 kCounterAlign;
+    const size_t partial_bytes =
+        n_split > 1 ? (size_t)n_q * dims->n_kv_heads * n_split * (32 + 16 * kHeadDim) * 4 : 0;
+    if (counter_bytes + partial_bytes > kScratchBytes) return QSA_ERR_WORKSPACE_TOO_SMALL;
+
+    void* base = nullptr;
+    if (scratch_address(&base) != cudaSuccess) return QSA_ERR_CUDA;
+    cudaStream_t st = (cudaStream_t)stream;
+    unsigned* counters = (unsigned*)base;
+    float* partial = (float*)((char*)base + counter_bytes);
+    if (n_split > 1 && cudaMemsetAsync(counters, 0, (size_t)n_q * dims->n_kv_heads * 4, st) != cudaSuccess)
+        return QSA_ERR_CUDA;
+    // no status word in this variant: out-of-range indices are still skipped, just not reported
+    const cudaError_t e = launch_attention(*dims, q, k_cache, v_cache, q_seq, q_pos, sel_idx, sel_cnt, n_q, out,
+                                           n_split, partial, counters, nullptr, st);
+    return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
+}

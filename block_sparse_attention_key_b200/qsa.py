@@ -31,6 +31,7 @@ QSA_MODE_PREFILL = 1
 EXPORTED = (
     "qsa_workspace_bytes", "qsa_workspace_init", "qsa_read_device_status", "qsa_status_string",
     "qsa_pool_block_keys", "qsa_index_scores", "qsa_topk_blocks", "qsa_sparse_attn", "qsa_forward",
+    "qsa_sparse_attn_noalloc",
 )
 
 
@@ -84,6 +85,7 @@ def load(path=LIB_PATH):
     L.qsa_topk_blocks.argtypes = [D, P, I64, P, I32, I64, P, P, P, SZ, P]
     L.qsa_sparse_attn.argtypes = [D, P, P, P, P, P, P, P, I32, P, P, SZ, P]
     L.qsa_forward.argtypes = [D, ctypes.POINTER(qsa_forward_args), P, SZ, P]
+    L.qsa_sparse_attn_noalloc.argtypes = [D, P, P, P, P, P, P, P, I32, P, P]
     for name in EXPORTED:
         if name not in ("qsa_workspace_bytes", "qsa_status_string"):
             getattr(L, name).restype = ctypes.c_int
@@ -167,6 +169,14 @@ def qsa_sparse_attn(dims, q, k_cache, v_cache, q_seq, q_pos, sel_idx, sel_cnt, n
         ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(q_seq), _ptr(q_pos), _ptr(sel_idx),
         _ptr(sel_cnt), n_q, _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream)))
+
+
+def qsa_sparse_attn_noalloc(dims, q, k_cache, v_cache, q_seq, q_pos, sel_idx, sel_cnt, n_q, out, stream=None):
+    """qsa_sparse_attn for callers that cannot allocate: scratch comes from a fixed
+    16 MiB array inside the library (see include/qsa.h)."""
+    _check("qsa_sparse_attn_noalloc", load().qsa_sparse_attn_noalloc(
+        ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(q_seq), _ptr(q_pos), _ptr(sel_idx),
+        _ptr(sel_cnt), n_q, _ptr(out), _stream(stream)))
 
 
 def qsa_forward(dims, *, q, k_cache, v_cache, idx_k, pooled, q_idx, w, len_before, len_after, q_seq, q_pos,

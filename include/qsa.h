@@ -150,6 +150,26 @@ int qsa_sparse_attn(const qsa_dims* dims, const void* q, const void* k_cache, co
                     const int32_t* sel_cnt, int32_t n_q, void* out, void* workspace,
                     size_t ws_bytes, void* stream);
 
+/* Step 4 without a caller workspace.  The pages describe nothing like it: it
+ * exists for callers that cannot allocate device memory — an engine whose
+ * allocator has already handed all of HBM to its KV cache, a frozen CUDA-graph
+ * memory plan, or a plain C host that only owns the tensors it passes — and so
+ * cannot provide qsa_sparse_attn's workspace.  Same arguments, layouts, math and
+ * results as qsa_sparse_attn, without workspace and ws_bytes.
+ * Scratch (split-K partials and completion counters) comes from a 16 MiB array
+ * built into the library; every GPU that loads the library holds it until the
+ * process exits.  A call needing more than that (roughly: more than 128 decode
+ * queries with 4 KV heads) returns QSA_ERR_WORKSPACE_TOO_SMALL before launching.
+ * The first call on each device, with that device current, looks the array's
+ * device address up (cudaGetSymbolAddress); make that first call before any
+ * stream capture.  All calls share the array: counters are cleared at the start
+ * of each call, and calls whose executions overlap on the GPU race on it.  No
+ * device status word: out-of-range indices are skipped but not reported.
+ * Nothing in this call allocates memory. */
+int qsa_sparse_attn_noalloc(const qsa_dims* dims, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,
+                            const int32_t* sel_cnt, int32_t n_q, void* out, void* stream);
+
 /* All inputs of one layer call (see the layouts above). */
 typedef struct qsa_forward_args {
     const void* q;            /* bf16 [n_q][n_q_heads][head_dim] */
