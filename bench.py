@@ -8,8 +8,8 @@ One process per GPU (torchrun for N > 1).  Every rank owns its own batch of
 sequences (independent problems: weak scaling, no data-path collective).  A step
 is the whole layer through the C ABI (qsa_forward): pool the appended token's
 block, score every complete causal block, select the top 512, gathered attention.
-Inputs sit in HBM when the timed region starts; L2 is flushed (a 512 MiB write)
-before every timed step and the flush is outside the timed events.  Rank 0 prints
+Inputs sit in HBM when the timed region starts; L2 is flushed (a 512 MiB write,
+then a 512 MiB read) before every timed step, outside the timed events.  Rank 0 prints
 one JSON line.  `--impl reference` times the CPU oracle on the same workload.
 """
 
@@ -55,7 +55,7 @@ def workload_config(wl):
             "context": max(st.len_after), "q_heads": wl.n_q_heads, "kv_heads": wl.n_kv_heads,
             "head_dim": wl.head_dim, "indexer": f"{wl.n_idx_heads}x{wl.idx_dim}", "block": wl.block_size,
             "top_k_blocks": wl.top_k, "steps_per_unit": len(wl.steps),
-            "l2": "flushed by a 512 MiB write before every timed step (outside the timed events)"}
+            "l2": "flushed before every timed step (512 MiB write, then 512 MiB read; outside the timed events)"}
 
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -252,22 +252,33 @@ def run_ours(args, wl):
     outs = [torch.empty((T["n_q"], wl.n_q_heads, wl.head_dim), dtype=torch.bfloat16, device="cuda") for T in steps]
     sels = [torch.empty((T["n_q"], wl.top_k), dtype=torch.int32, device="cuda") for T in steps]
     cnts = [torch.empty((T["n_q"],), dtype=torch.int32, device="cuda") for T in steps]
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    stream = torch.cuda.current_stream()
+    # L2 flush: write one buffer larger than L2, then read another, so L2 ends up
+    # full of clean lines that belong to neither the inputs nor the outputs
+    flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    flush_sink = torch.empty((), dtype=torch.float32, device="cuda")
+
+    def flush():
+        flush_w.fill_(1)
+        torch.sum(flush_r, dim=0, out=flush_sink)
+
+    def forward(T, out, sel, cnt, src=None):
+        src = src or T
+        qsa.qsa_forward(dims, q=src["q"], k_cache=dw.k_cache, v_cache=dw.v_cache, idx_k=dw.idx_k, pooled=dw.pooled,
+                        q_idx=src["q_idx"], w=src["w"], len_before=src["len_before"], len_after=src["len_after"],
+                        q_seq=src["q_seq"], q_pos=src["q_pos"], n_q=T["n_q"], max_new_tokens=T["max_new_tokens"],
+                        max_blocks=T["max_blocks"], mode=mode, out=out, workspace=ws, sel_idx=sel, sel_cnt=cnt)
 
     def unit():
         """One unit of work: every step of the workload (one step for most workloads)."""
         for T, out, sel, cnt in zip(steps, outs, sels, cnts):
-            qsa.qsa_forward(dims, q=T["q"], k_cache=dw.k_cache, v_cache=dw.v_cache, idx_k=dw.idx_k,
-                            pooled=dw.pooled, q_idx=T["q_idx"], w=T["w"], len_before=T["len_before"],
-                            len_after=T["len_after"], q_seq=T["q_seq"], q_pos=T["q_pos"], n_q=T["n_q"],
-                            max_new_tokens=T["max_new_tokens"], max_blocks=T["max_blocks"], mode=mode, out=out,
-                            workspace=ws, sel_idx=sel, sel_cnt=cnt, stream=stream)
+            forward(T, out, sel, cnt)
 
     def timed(fn, k):
+        stream = torch.cuda.current_stream()
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
         for a, b in evs:
-            flush.fill_(1)
+            flush()
             a.record(stream)
             fn()
             b.record(stream)
@@ -280,19 +291,27 @@ def run_ours(args, wl):
     flags = qsa.qsa_read_device_status(ws)
     if flags:
         raise SystemExit(f"device status flags {flags:#x} after warm-up")
+    # the step as a CUDA graph: all lengths and positions are device-side, so it replays as is
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        unit()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
 
     clocks = Clocks(local) if rank == 0 else None
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
-    ms = timed(unit, args.steps)
+    ms = timed(graph.replay, args.steps)
     torch.cuda.synchronize()
     barrier()
     wall = time.perf_counter() - wall0
     clk = clocks.stop() if clocks else None
     ms_per_step = max_over_ranks(sum(ms) / len(ms))
     value = world * n_q_unit / (ms_per_step / 1e3)
+    ms_eager = max_over_ranks(float(np.mean(timed(unit, args.steps))))
 
     # ---- per-kernel breakdown through the standalone entry points (same inputs) ----
     T = steps[-1]
@@ -300,24 +319,24 @@ def run_ours(args, wl):
     ld = (mb + 3) // 4 * 4
     scores = torch.empty((n_q, ld), dtype=torch.float32, device="cuda")
     out_k = torch.empty_like(outs[-1])
-    sel_k, cnt_k = sels[-1], cnts[-1]
+    sel_k, cnt_k = sels[-1].clone(), cnts[-1].clone()
     ws_k = torch.empty(qsa.qsa_workspace_bytes(dims, n_q, mb, 0), dtype=torch.uint8, device="cuda")
     qsa.qsa_workspace_init(ws_k)
     kernels = {}
     if mode == qsa.QSA_MODE_DECODE:
         run_score = lambda: qsa.qsa_index_scores(dims, T["q_idx"], T["w"], dw.pooled, T["q_seq"], T["q_pos"], n_q,
-                                                  mb, scores, ld, ws_k, stream=stream)
+                                                  mb, scores, ld, ws_k)
         run_score()
-        run_topk = lambda: qsa.qsa_topk_blocks(dims, scores, ld, T["q_pos"], n_q, mb, sel_k, cnt_k, ws_k,
-                                                stream=stream)
+        run_topk = lambda: qsa.qsa_topk_blocks(dims, scores, ld, T["q_pos"], n_q, mb, sel_k, cnt_k, ws_k)
         kernels["index_scores_us"] = 1e3 * float(np.mean(timed(run_score, args.steps)))
         kernels["topk_us"] = 1e3 * float(np.mean(timed(run_topk, args.steps)))
     run_attn = lambda: qsa.qsa_sparse_attn(dims, T["q"], dw.k_cache, dw.v_cache, T["q_seq"], T["q_pos"], sel_k,
-                                            cnt_k, n_q, out_k, ws_k, stream=stream)
+                                            cnt_k, n_q, out_k, ws_k)
     run_attn()
     attn_ms = float(np.mean(timed(run_attn, args.steps)))
     kernels["sparse_attn_us"] = 1e3 * attn_ms
     kernels["attn_matches_forward"] = bool(torch.equal(out_k, outs[-1]))
+    kernels["step_eager_us"] = 1e3 * ms_eager
 
     # algorithmic bytes of the gathered attention: K+V rows of every attended token
     # (4 per selected block plus the partial block) for every KV head, q in, out written
@@ -328,61 +347,72 @@ def run_ours(args, wl):
     hbm_peak, tc_peak, peak_kind = load_peaks()
     achieved = attn_bytes / (attn_ms / 1e3) / 1e9
     roofline = {"kernel": "k_sparse_attn", "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
-                "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "peak_source": f"{peak_kind} hbm_gbs (burst copy)",
-                "algorithmic_bytes_per_launch": attn_bytes,
-                "traffic": load_traffic("k_sparse_attn", wl.name)}
+                "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                "peak_source": f"{peak_kind} hbm_gbs (burst copy)",
+                "algorithmic_bytes_per_launch": attn_bytes, "traffic": load_traffic("k_sparse_attn", wl.name)}
 
     # ---- end to end: host buffers in, host buffer out, copies inside the timed region ----
-    host_in = []
+    # Every step's inputs travel in one pinned host buffer: queries, indexer inputs,
+    # positions, and the appended tokens' K/V rows and indexer keys, which are
+    # scattered into the caches on the device.
+    e2e_steps = []
     for si, T in enumerate(steps):
         st = wl.steps[si]
-        h = {k: T[k].cpu().pin_memory() for k in ("q", "q_idx", "w", "len_before", "len_after", "q_seq", "q_pos")}
-        # the appended token(s) of every sequence: K/V rows and indexer keys
-        h["new"] = [(s, a, b) for s, (a, b) in enumerate(zip(st.len_before, st.len_after)) if b > a]
-        h["k_new"] = [dw.k_cache[s, :, a:b].cpu().pin_memory() for s, a, b in h["new"]]
-        h["v_new"] = [dw.v_cache[s, :, a:b].cpu().pin_memory() for s, a, b in h["new"]]
-        h["ik_new"] = [dw.idx_k[s, a:b].cpu().pin_memory() for s, a, b in h["new"]]
-        host_in.append(h)
-    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
-    dev_in = [{k: torch.empty_like(T[k]) for k in ("q", "q_idx", "w", "len_before", "len_after", "q_seq", "q_pos")}
-              for T in steps]
-    h2d = sum(sum(h[k].numel() * h[k].element_size() for k in ("q", "q_idx", "w", "len_before", "len_after",
-                                                                "q_seq", "q_pos"))
-              + sum(x.numel() * x.element_size() for x in h["k_new"] + h["v_new"] + h["ik_new"]) for h in host_in)
-    d2h = sum(o.numel() * o.element_size() for o in host_out)
+        parts = {k: T[k] for k in ("q", "q_idx", "w", "len_before", "len_after", "q_seq", "q_pos")}
+        new = [(s, a, b) for s, (a, b) in enumerate(zip(st.len_before, st.len_after)) if b > a]
+        seq_i = torch.tensor([s for s, a, b in new for _ in range(a, b)], dtype=torch.int64, device="cuda")
+        pos_i = torch.tensor([p for s, a, b in new for p in range(a, b)], dtype=torch.int64, device="cuda")
+        parts["k_new"] = dw.k_cache[seq_i, :, pos_i].contiguous()
+        parts["v_new"] = dw.v_cache[seq_i, :, pos_i].contiguous()
+        parts["ik_new"] = dw.idx_k[seq_i, pos_i].contiguous()
+        layout, off = {}, 0
+        for k, v in parts.items():
+            nb = v.numel() * v.element_size()
+            layout[k] = (off, nb, v.dtype, tuple(v.shape))
+            off += (nb + 255) // 256 * 256
+        h_in = torch.empty(off, dtype=torch.uint8).pin_memory()
+        for k, v in parts.items():
+            o, nb, _, _ = layout[k]
+            h_in[o:o + nb].copy_(v.reshape(-1).view(torch.uint8).cpu())
+        d_in = torch.empty(off, dtype=torch.uint8, device="cuda")
+        view = {k: d_in[o:o + nb].view(dt).view(shape) for k, (o, nb, dt, shape) in layout.items()}
+        h_out = torch.empty(tuple(outs[si].shape), dtype=outs[si].dtype).pin_memory()
+        e2e_steps.append((T, h_in, d_in, view, seq_i, pos_i, h_out))
 
     def unit_e2e():
-        for si, (T, h, d, out, sel, cnt, ho) in enumerate(zip(steps, host_in, dev_in, outs, sels, cnts, host_out)):
-            for k in d:
-                d[k].copy_(h[k], non_blocking=True)
-            for (s, a, b), kn, vn, ikn in zip(h["new"], h["k_new"], h["v_new"], h["ik_new"]):
-                dw.k_cache[s, :, a:b].copy_(kn, non_blocking=True)
-                dw.v_cache[s, :, a:b].copy_(vn, non_blocking=True)
-                dw.idx_k[s, a:b].copy_(ikn, non_blocking=True)
-            qsa.qsa_forward(dims, q=d["q"], k_cache=dw.k_cache, v_cache=dw.v_cache, idx_k=dw.idx_k,
-                            pooled=dw.pooled, q_idx=d["q_idx"], w=d["w"], len_before=d["len_before"],
-                            len_after=d["len_after"], q_seq=d["q_seq"], q_pos=d["q_pos"], n_q=T["n_q"],
-                            max_new_tokens=T["max_new_tokens"], max_blocks=T["max_blocks"], mode=mode, out=out,
-                            workspace=ws, sel_idx=sel, sel_cnt=cnt, stream=stream)
-            ho.copy_(out, non_blocking=True)
-        stream.synchronize()
+        for (T, h_in, d_in, view, seq_i, pos_i, h_out), out, sel, cnt in zip(e2e_steps, outs, sels, cnts):
+            d_in.copy_(h_in, non_blocking=True)
+            dw.k_cache[seq_i, :, pos_i] = view["k_new"]
+            dw.v_cache[seq_i, :, pos_i] = view["v_new"]
+            dw.idx_k[seq_i, pos_i] = view["ik_new"]
+            forward(T, out, sel, cnt, src=view)
+            h_out.copy_(out, non_blocking=True)
 
     for _ in range(3):
         unit_e2e()
+    torch.cuda.synchronize()
+    graph_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_e2e):
+        unit_e2e()
     e2e_ms = []
     for _ in range(args.steps):
-        flush.fill_(1)
+        flush()
         torch.cuda.synchronize()
         t0 = time.perf_counter()
-        unit_e2e()
+        graph_e2e.replay()
+        torch.cuda.current_stream().synchronize()
         e2e_ms.append(1e3 * (time.perf_counter() - t0))
     e2e_ms = max_over_ranks(float(np.mean(e2e_ms)))
+    h2d = sum(x[1].numel() for x in e2e_steps)
+    d2h = sum(x[6].numel() * x[6].element_size() for x in e2e_steps)
     e2e = {"value": world * n_q_unit / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-           "timing": "host wall clock around copies in, qsa_forward, copy out, stream sync"}
+           "timing": "host wall clock around one CUDA-graph replay of: one H2D copy of the step's inputs from "
+                     "pinned memory, scatter of the appended K/V/indexer rows, qsa_forward, D2H copy of the "
+                     "output, stream sync"}
 
     flags = qsa.qsa_read_device_status(ws)
-    # our kernels per unit: pool (when tokens complete a block range), score, select x3, attention
+    # our kernels per unit: pool (when tokens are appended), score, select x3, attention
     launches_per_step = sum((1 if T["max_new_tokens"] > 0 else 0) + 4 + 1 for T in steps)
     if mode == qsa.QSA_MODE_PREFILL:
         rows = max(1, min(steps[0]["n_q"], (256 << 20) // (4 * max(1, steps[0]["max_blocks"]))))
@@ -391,7 +421,8 @@ def run_ours(args, wl):
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded SplitMix64 inputs, see DESIGN.md)",
-            "config": dict(workload_config(wl), parallelism=f"replicas x{world} (independent sequences per GPU)"),
+            "config": dict(workload_config(wl), parallelism=f"replicas x{world} (independent sequences per GPU)",
+                           execution="CUDA graph of the unit's qsa_forward calls"),
             "roofline": roofline, "kernels": kernels, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clk,
             "wall_s_timed_region": round(wall, 4), "device_status": flags}
@@ -399,6 +430,7 @@ def run_ours(args, wl):
         line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:
         print(json.dumps(line), flush=True)
+    del graph, graph_e2e
     if world > 1:
         dist.destroy_process_group()
 

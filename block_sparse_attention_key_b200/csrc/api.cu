@@ -80,8 +80,8 @@ WsLayout plan_workspace(const qsa_dims& d, int32_t n_q, int64_t max_blocks, int3
     L.ctrl = off + align_up((size_t)n_q * d.n_kv_heads * 4);
     L.ctrl_bytes = (L.ctrl - L.attn_cnt) + (size_t)rows * sizeof(TopkCtrl);
     off = L.attn_cnt + align_up(L.ctrl_bytes);
-    L.lh3 = off;
-    off += align_up((size_t)rows * L.n_chunks * kBins3 * 4);
+    L.cand = off;
+    off += align_up((size_t)rows * kCandCap * 8);
     L.tmp = off;
     off += align_up((size_t)rows * kTopK * 4);
     L.score_ld = (max_blocks + 3) / 4 * 4;
@@ -196,7 +196,7 @@ int qsa_topk_blocks(const qsa_dims* dims, const float* scores, int64_t ld_scores
     cudaError_t e = cudaMemsetAsync(ws + L.attn_cnt, 0, L.ctrl_bytes, st);
     if (e != cudaSuccess) return QSA_ERR_CUDA;
     return cuda_status(launch_topk(scores, ld_scores, q_pos, 0, n_q, max_blocks, dims->kv_capacity, L.chunk,
-                                   L.n_chunks, (TopkCtrl*)(ws + L.ctrl), (unsigned*)(ws + L.lh3),
+                                   L.n_chunks, (TopkCtrl*)(ws + L.ctrl), (unsigned long long*)(ws + L.cand),
                                    (int32_t*)(ws + L.tmp), sel_idx, sel_cnt, false, (unsigned*)ws, st));
 }
 
@@ -269,18 +269,22 @@ int qsa_forward(const qsa_dims* dims, const qsa_forward_args* a, void* workspace
         // scoring + selection in batches of L.score_rows rows (all rows at once in decode)
         for (int32_t row0 = 0; row0 < n_q; row0 += L.score_rows) {
             const int32_t n = n_q - row0 < L.score_rows ? n_q - row0 : L.score_rows;
-            e = cudaMemsetAsync(ws + L.ctrl, 0, (size_t)n * sizeof(TopkCtrl), st);
+            if (row0 == 0 && n == n_q)  // one batch: clear split counters and control blocks together
+                e = cudaMemsetAsync(ws + L.attn_cnt, 0, L.ctrl_bytes, st);
+            else
+                e = cudaMemsetAsync(ws + L.ctrl, 0, (size_t)n * sizeof(TopkCtrl), st);
             if (e != cudaSuccess) return QSA_ERR_CUDA;
             e = launch_score_decode(*dims, a->q_idx, a->w, a->pooled, a->q_seq, a->q_pos, row0, n, a->max_blocks,
                                     scores, L.score_ld, L.chunk, ctrl, status, st);
             if (e != cudaSuccess) return QSA_ERR_CUDA;
             e = launch_topk(scores, L.score_ld, a->q_pos, row0, n, a->max_blocks, dims->kv_capacity, L.chunk,
-                            L.n_chunks, ctrl, (unsigned*)(ws + L.lh3), (int32_t*)(ws + L.tmp), sel_idx, sel_cnt,
+                            L.n_chunks, ctrl, (unsigned long long*)(ws + L.cand), (int32_t*)(ws + L.tmp), sel_idx,
+                            sel_cnt,
                             true, status, st);
             if (e != cudaSuccess) return QSA_ERR_CUDA;
         }
     }
-    if (L.n_split > 1) {
+    if (L.n_split > 1 && !(a->max_blocks > 0 && L.score_rows == n_q)) {
         e = cudaMemsetAsync(ws + L.attn_cnt, 0, (size_t)n_q * dims->n_kv_heads * 4, st);
         if (e != cudaSuccess) return QSA_ERR_CUDA;
     }

@@ -336,11 +336,13 @@ k_sparse_attn(const uint4* __restrict__ q, const uint16_t* __restrict__ k_cache,
     if (row >= G) return;
     const float* base = partial + pair * n_split * pstride;
     float Mg = -INFINITY;
+#pragma unroll 8
     for (int sp = 0; sp < n_split; ++sp) Mg = fmaxf(Mg, __ldcg(base + sp * pstride + row));
     const float Mgu = Mg == -INFINITY ? 0.f : Mg;
     float Lg = 0.f, og[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) og[e] = 0.f;
+#pragma unroll 4
     for (int sp = 0; sp < n_split; ++sp) {
         const float* ps = base + sp * pstride;
         const float f = exp2f(__ldcg(ps + row) - Mgu);
@@ -389,8 +391,15 @@ cudaError_t launch_attention(const qsa_dims& d, const void* q, const void* k_cac
     const int bps_tiles = ((bps + kTileBlocks - 1) / kTileBlocks) * kTileBlocks;
     const float scale = d.softmax_scale > 0.f ? d.softmax_scale : 1.0f / sqrtf((float)d.head_dim);
     const float scale_log2 = scale * 1.4426950408889634f;
-    cudaError_t e = cudaFuncSetAttribute(k_sparse_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
-    if (e != cudaSuccess) return e;
+    static bool attr_set[128] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 128 && !attr_set[dev]) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(k_sparse_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
     dim3 grid((unsigned)n_split, (unsigned)d.n_kv_heads, (unsigned)n_q);
     k_sparse_attn<<<grid, kThreads, kSmemTotal, st>>>(
         (const uint4*)q, (const uint16_t*)k_cache, (const uint16_t*)v_cache, q_seq, q_pos, sel_idx, sel_cnt,

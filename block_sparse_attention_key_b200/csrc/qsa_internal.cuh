@@ -22,6 +22,7 @@ constexpr int kMaxGroup = 16;    // query heads per KV head handled by one atten
 constexpr int kBins1 = 4096;
 constexpr int kBins2 = 4096;
 constexpr int kBins3 = 256;
+constexpr int kCandCap = 4096;  // boundary-bin candidates finished in shared memory
 
 enum SelectMode : int {
     kSelUndecided = 0,  // more digits needed
@@ -42,7 +43,9 @@ struct TopkCtrl {
     int need;              // entries still to take from keys equal to `prefix`
     int mode;              // SelectMode
     int n_cand;            // n_c of the query (after the max_blocks cut)
-    unsigned pad[6];
+    unsigned bin_count;    // keys in the bin of the last resolved digit
+    unsigned ncand;        // entries appended to the candidate list
+    unsigned pad[4];
 };
 static_assert(sizeof(TopkCtrl) % 64 == 0, "TopkCtrl keeps 64-byte alignment");
 
@@ -69,8 +72,8 @@ struct WsLayout {
     size_t ctrl = 0;       // TopkCtrl[n_q] then attention counters u32[n_q * n_kv_heads]
     size_t ctrl_bytes = 0; // bytes zeroed at the start of each select/attention
     size_t attn_cnt = 0;   // offset of the attention split counters (inside ctrl)
-    size_t lh3 = 0;        // u32 [n_q][n_chunks][256] per-chunk digit-3 histograms
-    size_t tmp = 0;        // i32 [n_q][top_k] unordered selection
+    size_t cand = 0;       // u64 [rows][kCandCap] boundary-bin candidates (key << 32 | block)
+    size_t tmp = 0;        // i32 [rows][top_k] unordered winners
     size_t scores = 0;     // f32 [n_rows][ld] decode score rows
     int64_t score_ld = 0;
     int32_t score_rows = 0;
@@ -103,9 +106,9 @@ cudaError_t launch_score_decode(const qsa_dims& d, const void* q_idx, const floa
 // Radix select over score rows [0, n_rows) (query i = row0 + r).  If `hist_done`
 // the digit-1 histogram was built by the scoring kernel.
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, int32_t row0, int32_t n_rows,
-                        int64_t max_blocks, int64_t kv_capacity, int chunk, int n_chunks, TopkCtrl* ctrl, unsigned* lh3,
-                        int32_t* tmp, int32_t* sel_idx, int32_t* sel_cnt, bool hist_done, unsigned* status,
-                        cudaStream_t st);
+                        int64_t max_blocks, int64_t kv_capacity, int chunk, int n_chunks, TopkCtrl* ctrl,
+                        unsigned long long* cand, int32_t* tmp, int32_t* sel_idx, int32_t* sel_cnt, bool hist_done,
+                        unsigned* status, cudaStream_t st);
 
 cudaError_t launch_attention(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,
                              const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,

@@ -8,15 +8,31 @@
 // over the complete causal blocks b < floor((t+1)/4).
 //
 // A decode query touches every pooled key of its sequence once (128 B each), so
-// this is an HBM stream: 4 lanes share a block (16 dims = two 16-byte loads each),
-// every thread has 4 blocks (8 loads) in flight, and a 4x4 transpose-reduce over
-// the lane quad leaves each lane with the 4 head sums of one block, whose score it
-// writes.  fp32 accumulation of bf16 x bf16 products (exact for small integers).
+// this is an HBM stream: 4 lanes share a block (16 dims, two 16-byte pieces each).
+// Each thread stages its own pieces with cp.async into a private shared-memory
+// ring two rounds deep (8 x 16 B per round, 64 KiB in flight per CTA), and a 4x4
+// transpose-reduce over the lane quad leaves each lane with the 4 head sums of one
+// block, whose score it writes.  fp32 accumulation of bf16 x bf16 products (exact for small integers).
 // Optionally the same pass histograms the scores' top key digit for the select.
 
 #include "select_common.cuh"
 
 namespace qsa {
+
+namespace {
+
+constexpr int kRounds = 2;                                 // rounds of 256 blocks in flight per CTA
+constexpr int kStageBytes = kRounds * 4 * 2 * 256 * 16;     // 64 KiB of dynamic shared memory
+
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* g, int src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(saddr), "l"(g), "r"(src_bytes));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+}  // namespace
 
 template <bool kHist>
 __global__ void __launch_bounds__(256, 2)
@@ -25,6 +41,8 @@ k_score_decode(const uint4* __restrict__ q_idx, const float* __restrict__ w, con
                int32_t batch, int64_t kv_capacity, int64_t max_blocks, float* __restrict__ scores,
                int64_t ld, int chunk, TopkCtrl* __restrict__ ctrl, unsigned* status)
 {
+    // per-thread private staging: [round][u][half][thread] x 16 B (conflict-free 16-byte lane stride)
+    extern __shared__ __align__(16) uint4 s_stage[];
     __shared__ unsigned s_hist[kHist ? kBins1 : 1];
     __shared__ unsigned s_warp[8];
     __shared__ int s_last;
@@ -57,6 +75,29 @@ k_score_decode(const uint4* __restrict__ q_idx, const float* __restrict__ w, con
     const int sub = tid & 3;   // this lane's 16-dim slice
 
     if (b0 < b_valid) {
+        const uint4* prow = pooled + (int64_t)s * (kv_capacity / kBlock) * 8 + 2 * sub;
+        const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(s_stage);
+        const int n_rounds = (int)((b_valid - b0 + 255) / 256);
+        // stage round `rd` of this thread's 4 blocks (two 16-byte halves each)
+        auto issue = [&](int rd) {
+            const int slot = rd % kRounds;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int64_t b = b0 + (int64_t)rd * 256 + grp + 64 * u;
+                const bool in = b < b_valid;
+                const uint4* src = in ? prow + b * 8 : prow;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf)
+                    cp_async16(sbase + (uint32_t)((((slot * 4 + u) * 2 + hf) * 256 + tid) * 16), src + hf,
+                               in ? 16 : 0);
+            }
+        };
+#pragma unroll
+        for (int rd = 0; rd < kRounds - 1; ++rd) {
+            if (rd < n_rounds) issue(rd);
+            cp_async_commit();
+        }
+
         float qf[kIdxHeads][16];
 #pragma unroll
         for (int h = 0; h < kIdxHeads; ++h) {
@@ -72,28 +113,19 @@ k_score_decode(const uint4* __restrict__ q_idx, const float* __restrict__ w, con
         float wv[kIdxHeads];
 #pragma unroll
         for (int h = 0; h < kIdxHeads; ++h) wv[h] = __ldg(w + (int64_t)i * kIdxHeads + h);
-
-        const uint4* prow = pooled + (int64_t)s * (kv_capacity / kBlock) * 8 + 2 * sub;
         const bool odd = sub & 1, high = sub & 2;
 
-        for (int64_t base = b0; base < b_valid; base += 256) {
-            uint4 raw[4][2];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int64_t b = base + grp + 64 * u;
-                if (b < b_valid) {
-                    raw[u][0] = __ldg(prow + b * 8);
-                    raw[u][1] = __ldg(prow + b * 8 + 1);
-                } else {
-                    raw[u][0] = make_uint4(0, 0, 0, 0);
-                    raw[u][1] = make_uint4(0, 0, 0, 0);
-                }
-            }
+        for (int rd = 0; rd < n_rounds; ++rd) {
+            if (rd + kRounds - 1 < n_rounds) issue(rd + kRounds - 1);
+            cp_async_commit();
+            cp_async_wait<kRounds - 1>();  // this thread's copies of round rd have landed
+            const int slot = rd % kRounds;
             float acc[4][kIdxHeads];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const uint32_t x[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
-                                       raw[u][1].x, raw[u][1].y, raw[u][1].z, raw[u][1].w};
+                const uint4 lo = s_stage[((slot * 4 + u) * 2 + 0) * 256 + tid];
+                const uint4 hi = s_stage[((slot * 4 + u) * 2 + 1) * 256 + tid];
+                const uint32_t x[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
                 float p[16];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
@@ -124,12 +156,17 @@ k_score_decode(const uint4* __restrict__ q_idx, const float* __restrict__ w, con
                 const float mine = (high ? kb[h] : ka[h]) + __shfl_xor_sync(0xffffffffu, send, 2);
                 score = fmaf(wv[h], fmaxf(mine, 0.f), score);
             }
-            const int64_t b = base + grp + 64 * sub;
-            if (b < b_valid) {
-                srow[b] = score;
-                if (kHist) atomicAdd(&s_hist[orderable_key(score) >> 20], 1u);
+            const int64_t b = b0 + (int64_t)rd * 256 + grp + 64 * sub;
+            const bool in = b < b_valid;
+            if (in) srow[b] = score;
+            if (kHist) {
+                // one shared-memory atomic per distinct bin per warp
+                const unsigned bin = in ? orderable_key(score) >> 20 : 0xFFFFFFFFu;
+                const unsigned peers = __match_any_sync(0xffffffffu, bin);
+                if (in && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&s_hist[bin], (unsigned)__popc(peers));
             }
         }
+        cp_async_wait<0>();
     }
     if (!kHist) return;
 
@@ -156,12 +193,24 @@ cudaError_t launch_score_decode(const qsa_dims& d, const void* q_idx, const floa
     if (n_rows <= 0 || max_blocks <= 0) return cudaSuccess;
     const int64_t n_chunks = (max_blocks + chunk - 1) / chunk;
     dim3 grid((unsigned)n_chunks, (unsigned)n_rows);
+    static bool attr_set[128] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 128 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(k_score_decode<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kStageBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(k_score_decode<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kStageBytes);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
     if (ctrl)
-        k_score_decode<true><<<grid, 256, 0, st>>>((const uint4*)q_idx, w, (const uint4*)pooled, q_seq, q_pos,
+        k_score_decode<true><<<grid, 256, kStageBytes, st>>>((const uint4*)q_idx, w, (const uint4*)pooled, q_seq, q_pos,
                                                    row0, d.batch, d.kv_capacity, max_blocks, scores, ld,
                                                    chunk, ctrl, status);
     else
-        k_score_decode<false><<<grid, 256, 0, st>>>((const uint4*)q_idx, w, (const uint4*)pooled, q_seq, q_pos,
+        k_score_decode<false><<<grid, 256, kStageBytes, st>>>((const uint4*)q_idx, w, (const uint4*)pooled, q_seq, q_pos,
                                                     row0, d.batch, d.kv_capacity, max_blocks, scores, ld,
                                                     chunk, nullptr, status);
     return cudaGetLastError();

@@ -52,33 +52,43 @@ __device__ __forceinline__ int block_rank_256(bool p, int* s_cnt /*[8]*/, int* t
 }
 
 // Fix the next digit of the threshold key.  Run by all 256 threads of the CTA
-// that completed a histogram pass.  `hist` (global, nbins = 256 * per) counts
-// the candidates whose key matches the resolved prefix, by their next digit.
-// Among them the top `need` are wanted.  Updates ctrl->{prefix, nbits, need, mode}.
-__device__ __forceinline__ void resolve_digit(TopkCtrl* ctrl, const unsigned* hist, int per, int bits,
-                                              bool final_digit, unsigned prefix, int nbits, int need,
-                                              unsigned* s_warp)
+// that completed a histogram pass.  `hist` (global, 256 * kPer bins) counts the
+// candidates whose key matches the resolved prefix, by their next digit.  Among
+// them the top `need` are wanted.  Updates ctrl->{prefix, nbits, need, mode}.
+// Each thread owns kPer consecutive bins, loaded once (independent loads).
+template <int kPer>
+__device__ __forceinline__ void resolve_digit(TopkCtrl* ctrl, const unsigned* hist, int bits, bool final_digit,
+                                              unsigned prefix, int nbits, int need, unsigned* s_warp)
 {
     const int tid = threadIdx.x;
+    unsigned h[kPer];
     unsigned local = 0;
-    for (int k = 0; k < per; ++k) local += __ldcg(hist + tid * per + k);
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) h[k] = __ldcg(hist + tid * kPer + k);
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) local += h[k];
     const unsigned suf = block_suffix_sum_256(local, s_warp);
     const unsigned after = suf - local;
     if (suf >= (unsigned)need && after < (unsigned)need) {
         unsigned run = after;
-        for (int k = per - 1; k >= 0; --k) {
-            const unsigned h = __ldcg(hist + tid * per + k);
-            if (run + h >= (unsigned)need) {
-                const unsigned digit = (unsigned)(tid * per + k);
-                const int need_here = need - (int)run;
-                ctrl->prefix = (prefix << bits) | digit;
-                ctrl->nbits = nbits + bits;
-                ctrl->need = need_here;
-                ctrl->mode = (h == (unsigned)need_here) ? kSelPrefix : (final_digit ? kSelTies : kSelUndecided);
-                break;
+        int found = -1;
+        unsigned found_h = 0, found_run = 0;
+#pragma unroll
+        for (int k = kPer - 1; k >= 0; --k) {
+            if (found < 0 && run + h[k] >= (unsigned)need) {
+                found = k;
+                found_h = h[k];
+                found_run = run;
             }
-            run += h;
+            run += h[k];
         }
+        const unsigned digit = (unsigned)(tid * kPer + found);
+        const int need_here = need - (int)found_run;
+        ctrl->prefix = (prefix << bits) | digit;
+        ctrl->nbits = nbits + bits;
+        ctrl->need = need_here;
+        ctrl->bin_count = found_h;
+        ctrl->mode = (found_h == (unsigned)need_here) ? kSelPrefix : (final_digit ? kSelTies : kSelUndecided);
     }
 }
 
@@ -101,7 +111,7 @@ __device__ __forceinline__ void finish_digit1(TopkCtrl* ctrl, int64_t n_c, unsig
         return;
     }
     if (threadIdx.x == 0) ctrl->n_cand = (int)n_c;
-    resolve_digit(ctrl, ctrl->hist1, kBins1 / 256, 12, false, 0u, 0, kTopK, s_warp);
+    resolve_digit<kBins1 / 256>(ctrl, ctrl->hist1, 12, false, 0u, 0, kTopK, s_warp);
 }
 
 }  // namespace qsa

@@ -138,7 +138,7 @@ def _run_topk(score_rows, positions, max_blocks):
 
 def test_topk_matches_oracle_on_ties_and_ragged_counts():
     rng = np.random.default_rng(17)
-    n_cs = [0, 1, 511, 512, 513, 700, 5000, 20000, 20000, 20000, 20000, 3]
+    n_cs = [0, 1, 511, 512, 513, 700, 5000, 20000, 20000, 20000, 20000, 3, 20000, 20000, 16000]
     rows = [
         rng.integers(0, 4, n_cs[0]), rng.integers(0, 4, 1), rng.integers(0, 9, 511), rng.integers(0, 3, 512),
         rng.integers(0, 3, 513), rng.normal(size=700), rng.integers(0, 50, 5000) * 0.25,
@@ -147,6 +147,12 @@ def test_topk_matches_oracle_on_ties_and_ragged_counts():
         np.linspace(0, 1, 20000)[::-1].copy(),             # strictly decreasing: first 512
         np.where(rng.random(20000) < 0.5, -0.0, 0.0),      # signed zeros compare equal
         np.array([1.0, 1.0, 1.0]),
+        # 3,000 keys equal at the cut inside a small boundary bin: ordered re-scan path
+        np.where(np.arange(20000) % 6 == 1, 5.0, np.where(np.arange(20000) % 200 == 3, 10.0, 0.0)),
+        # 600 keys equal at the cut: pairwise index ranking of the ties
+        np.where(np.arange(20000) % 33 == 7, 5.0, np.where(np.arange(20000) % 97 == 3, 10.0, 1.0)),
+        # quarter-integer scores like the indexer's, many ties everywhere
+        rng.integers(0, 1200, 16000) * 0.25,
     ]
     rows = [np.asarray(r, dtype=np.float32) for r in rows]
     positions = [4 * c for c in n_cs]  # n_c(t) = c exactly (one partial token)
