@@ -11,7 +11,6 @@ namespace qsa {
 namespace {
 
 constexpr size_t kAlign = 256;
-constexpr int64_t kPrefillScoreBytes = 256ll << 20;  // score rows per prefill batch
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -39,15 +38,6 @@ int check_rows(const qsa_dims* d, int32_t n_q, int64_t max_blocks)
     return QSA_OK;
 }
 
-int32_t prefill_rows(int32_t n_q, int64_t max_blocks)
-{
-    const int64_t per = (max_blocks > 0 ? max_blocks : 1) * 4;
-    int64_t r = kPrefillScoreBytes / per;
-    if (r < 1) r = 1;
-    if (r > n_q) r = n_q;
-    return (int32_t)r;
-}
-
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA; }
 
 }  // namespace
@@ -69,7 +59,8 @@ WsLayout plan_workspace(const qsa_dims& d, int32_t n_q, int64_t max_blocks, int3
 {
     WsLayout L;
     size_t off = kAlign;  // status word
-    const int32_t rows = max_blocks > 0 ? (mode == QSA_MODE_PREFILL ? prefill_rows(n_q, max_blocks) : n_q) : 0;
+    // decode rows go through the score-row select; prefill chunks through the tensor-core path
+    const int32_t rows = (max_blocks > 0 && mode == QSA_MODE_DECODE) ? n_q : 0;
     L.score_rows = rows;
     L.chunk = select_chunk(max_blocks, rows);
     L.n_chunks = max_blocks > 0 ? (int)((max_blocks + L.chunk - 1) / L.chunk) : 0;
@@ -91,6 +82,20 @@ WsLayout plan_workspace(const qsa_dims& d, int32_t n_q, int64_t max_blocks, int3
     off += align_up((size_t)n_q * kTopK * 4 + (size_t)n_q * 4);
     L.partial = off;
     if (L.n_split > 1) off += align_up((size_t)n_q * d.n_kv_heads * L.n_split * (32 + 16 * kHeadDim) * 4);
+    if (mode == QSA_MODE_PREFILL && max_blocks > 0 && n_q > 0) {
+        L.pf_split = prefill_splits(n_q, max_blocks);
+        const size_t segs = (size_t)n_q * 2 * L.pf_split;
+        L.pf_cand = off;
+        off += align_up(segs * prefill_seg_cap() * 8);
+        L.pf_cnt = off;
+        off += align_up(segs * 4);
+        L.pf_theta = off;                 // thresholds, then the worklist count: zeroed together
+        L.pf_work = off + (size_t)n_q * 4;
+        off += align_up((size_t)(2 * n_q + 1) * 4);
+        L.pf_fb_ctas = n_q < 64 ? n_q : 64;
+        L.pf_scratch = off;
+        off += align_up((size_t)L.pf_fb_ctas * max_blocks * 4);
+    }
     L.total = off;
     return L;
 }
@@ -265,8 +270,16 @@ int qsa_forward(const qsa_dims* dims, const qsa_forward_args* a, void* workspace
         e = cudaMemsetAsync(sel_idx, 0xFF, (size_t)n_q * kTopK * 4, st);
         if (e == cudaSuccess) e = cudaMemsetAsync(sel_cnt, 0, (size_t)n_q * 4, st);
         if (e != cudaSuccess) return QSA_ERR_CUDA;
+    } else if (a->mode == QSA_MODE_PREFILL) {
+        e = cudaMemsetAsync(ws + L.pf_theta, 0, (size_t)(n_q + 1) * 4, st);
+        if (e != cudaSuccess) return QSA_ERR_CUDA;
+        e = launch_prefill_select(*dims, a->q_idx, a->w, a->pooled, a->q_seq, a->q_pos, n_q, a->max_blocks,
+                                  L.pf_split, (unsigned long long*)(ws + L.pf_cand), (unsigned*)(ws + L.pf_cnt),
+                                  (unsigned*)(ws + L.pf_theta), (int32_t*)(ws + L.pf_work),
+                                  (float*)(ws + L.pf_scratch), L.pf_fb_ctas, sel_idx, sel_cnt, status, st);
+        if (e != cudaSuccess) return QSA_ERR_CUDA;
     } else {
-        // scoring + selection in batches of L.score_rows rows (all rows at once in decode)
+        // decode: scoring + selection of all rows at once
         for (int32_t row0 = 0; row0 < n_q; row0 += L.score_rows) {
             const int32_t n = n_q - row0 < L.score_rows ? n_q - row0 : L.score_rows;
             if (row0 == 0 && n == n_q)  // one batch: clear split counters and control blocks together

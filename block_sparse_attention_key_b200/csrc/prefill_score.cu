@@ -1,0 +1,581 @@
+// Prefill indexer scoring and top-512 selection on the tcgen05 tensor cores
+// (steps 2 and 3 of the QSA layer for a chunk of queries of one sequence).
+//
+// blog.cecily.jp/6295 (Raschka's explainer paragraph) and keieiax.jp glossary
+// "Qwen Sparse Attention" (section on 4-token micro-blocks): every query scores
+// every complete causal block with a light indexer and keeps the best 512.  For a
+// chunk of queries this is a dense contraction: per 128-query tile and indexer
+// head h, S_h = Q_h (128 x 64) . P^T (64 x N) over the pooled keys P, then
+// score = sum_h w_h ReLU(S_h).  The score matrix (8 GiB at 8,192 queries x 1M
+// tokens) is never stored: each CTA streams its range of pooled keys and keeps,
+// per query row, only the blocks that can still be in the row's top 512.
+//
+// CTA = 10 warps, one CTA per SM (512 TMEM columns):
+//   warp 0      TMA producer: the 4 query tiles once, then 64-block pooled tiles
+//               (8 KiB, 128-byte swizzle) into an 8-deep ring;
+//   warp 1      TMEM allocator and MMA issuer: per pooled tile, 4 heads x 4 K-steps of
+//               tcgen05.mma (M=128, N=64, K=16, bf16 -> f32) into one of two
+//               accumulator stages (4 heads x 64 columns each);
+//   warps 2..9  epilogue, two warpgroups; each thread owns one query row (its TMEM
+//               lane) and half the columns of every tile: tcgen05.ld, ReLU, weights,
+//               head sum, causal cut, and a streaming admission test.
+// Admission: a row keeps every block whose score is at least its threshold.  The
+// threshold starts below every finite score and rises as the row's admitted
+// scores fill a 64-bin histogram (1/16-octave bins of the order-preserving key):
+// once 512 admitted blocks lie at or above a bin edge, no later block below that
+// edge can reach the top 512, and (as blocks arrive in increasing index order) a
+// later block equal to the edge loses every tie, so the thread's own cut is strict.
+// Thresholds are shared (non-strictly) with the other warpgroup through shared
+// memory and with other CTAs of the row through a global atomic max.  Admitted
+// (key, block) pairs are appended to per-(row, CTA, warpgroup) segments in global
+// memory; a finishing kernel selects the exact top 512 among them.
+//
+// All waits are bounded (a global-timer limit); on a timeout the kernel records
+// QSA_DEV_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
+
+#include <cfloat>
+
+#include <cudaTypedefs.h>
+
+#include "select_finish.cuh"
+#include "sm100_ptx.cuh"
+
+namespace qsa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kM = 128;                 // query rows per CTA
+constexpr int kN = 64;                  // pooled blocks per tile
+constexpr int kNumB = 8;                // pooled-tile ring depth
+constexpr int kEpiWarps = 8;
+constexpr int kK3Threads = 64 + 32 * kEpiWarps;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kHistBins = 64;
+constexpr int kHistShift = 19;          // 1/16-octave bins of the orderable key
+constexpr int kRaiseEvery = 32;         // admissions between threshold updates
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any single wait
+
+struct __align__(1024) K3Smem {
+    __nv_bfloat16 a[kIdxHeads][kM * kIdxDim];   // 4 x 16 KiB
+    __nv_bfloat16 b[kNumB][kN * kIdxDim];       // 8 x 8 KiB
+    uint32_t hist[2][kHistBins][kM];            // 64 KiB
+    float theta[2][kM];                         // published (non-strict) thresholds
+    float w[kM][kIdxHeads];
+    int n_c[kM];
+    uint64_t full[kNumB], empty[kNumB];
+    uint64_t tmem_full[2], tmem_empty[2];
+    uint64_t a_full, mma_done;
+    uint32_t tmem_base;
+    int error;
+    int nc_min, nc_max, seq;
+};
+
+__device__ __forceinline__ uint64_t now_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait: polls until the phase completes, the CTA's error flag is set, or
+// kWaitNs passes (then sets the flag).  Returns true only if the phase completed.
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volatile int* error, unsigned* status)
+{
+    const uint64_t t0 = now_ns();
+    for (uint32_t i = 0;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 63u) {
+            if (*error) return false;
+            if (now_ns() - t0 > kWaitNs) {
+                *error = 1;
+                set_status(status, QSA_DEV_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ float key_to_float(unsigned k)
+{
+    return __uint_as_float((k & 0x80000000u) ? (k ^ 0x80000000u) : ~k);
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kK3Threads, 1)
+k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_p,
+                    const float* __restrict__ w, const int32_t* __restrict__ q_seq,
+                    const int32_t* __restrict__ q_pos, int32_t n_q, int32_t batch, int64_t kv_capacity,
+                    int64_t max_blocks, int n_split, int seg_cap, unsigned long long* __restrict__ cand,
+                    unsigned* __restrict__ cand_cnt, unsigned* __restrict__ theta_g, unsigned* status)
+{
+    extern __shared__ uint8_t smem_raw[];
+    K3Smem& S = *reinterpret_cast<K3Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int split = blockIdx.x, mtile = blockIdx.y;
+    const int64_t row0 = (int64_t)mtile * kM;
+
+    // ---- setup: barriers, row metadata, TMEM ----
+    if (tid == 0) {
+        for (int i = 0; i < kNumB; ++i) {
+            mbar_init(&S.full[i], 1);
+            mbar_init(&S.empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&S.tmem_full[i], 1);
+            mbar_init(&S.tmem_empty[i], kEpiWarps);
+        }
+        mbar_init(&S.a_full, 1);
+        mbar_init(&S.mma_done, 1);
+        S.error = 0;
+        S.nc_min = INT_MAX;
+        S.nc_max = 0;
+        S.seq = q_seq[row0];
+        fence_mbar_init();
+    }
+    for (int k = tid; k < 2 * kHistBins * kM; k += kK3Threads) (&S.hist[0][0][0])[k] = 0;
+    __syncthreads();
+    if (tid < kM) {
+        const int64_t r = row0 + tid;
+        int nc = 0;
+        if (r < n_q) {
+            const int s = q_seq[r], t = q_pos[r];
+            const bool ok = s == S.seq && s >= 0 && s < batch && t >= 0 && (int64_t)t < kv_capacity;
+            if (!ok && split == 0) set_status(status, s != S.seq ? QSA_DEV_BAD_SEQ : QSA_DEV_BAD_POS);
+            if (ok) {
+                int64_t c = ((int64_t)t + 1) / kBlock;
+                if (c > max_blocks) {
+                    if (split == 0) set_status(status, QSA_DEV_BLOCKS_OVER);
+                    c = max_blocks;
+                }
+                nc = (int)c;
+            }
+#pragma unroll
+            for (int h = 0; h < kIdxHeads; ++h) S.w[tid][h] = w[r * kIdxHeads + h];
+        }
+        S.n_c[tid] = nc;
+        S.theta[0][tid] = S.theta[1][tid] = -FLT_MAX;
+        if (r < n_q) {
+            atomicMin(&S.nc_min, nc);
+            atomicMax(&S.nc_max, nc);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(&S.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // this CTA's range of pooled blocks: a 1/n_split share of the tile's longest row
+    const int nc_max = S.nc_max;
+    const int chunk = (((nc_max + n_split - 1) / n_split) + kN - 1) / kN * kN;
+    const int blk0 = split * chunk;
+    const int blk1 = min(blk0 + chunk, nc_max);
+    const int n_stages = blk1 > blk0 ? (blk1 - blk0 + kN - 1) / kN : 0;
+    const uint32_t tmem = S.tmem_base;
+    volatile int* err = &S.error;
+    const int64_t prow0 = (int64_t)S.seq * (kv_capacity / kBlock);
+
+    if (warp == 0) {
+        if (lane == 0 && n_stages > 0) {
+            prefetch_tensormap(&tmap_q);
+            prefetch_tensormap(&tmap_p);
+            mbar_arrive_expect_tx(&S.a_full, kIdxHeads * kM * kIdxDim * 2);
+            for (int h = 0; h < kIdxHeads; ++h) tma_load_3d(S.a[h], &tmap_q, &S.a_full, 0, h, (int)row0);
+            int issued = 0;
+            for (int j = 0; j < n_stages; ++j) {
+                const int slot = j % kNumB;
+                if (j >= kNumB && !wait_phase(&S.empty[slot], ((j / kNumB) - 1) & 1, err, status)) break;
+                mbar_arrive_expect_tx(&S.full[slot], kN * kIdxDim * 2);
+                tma_load_2d(S.b[slot], &tmap_p, &S.full[slot], 0, (int)(prow0 + blk0 + (int64_t)j * kN));
+                issued = j + 1;
+            }
+            if (*err) {
+                // drain: every issued tile and the query tiles must land before the CTA exits
+                wait_phase(&S.a_full, 0, err, status);
+                for (int j = max(0, issued - kNumB); j < issued; ++j) {
+                    const uint64_t t0 = now_ns();
+                    while (!mbar_try_wait(&S.full[j % kNumB], (j / kNumB) & 1) && now_ns() - t0 < kWaitNs) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && n_stages > 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(kM, kN);
+            uint64_t adesc[kIdxHeads];
+#pragma unroll
+            for (int h = 0; h < kIdxHeads; ++h) adesc[h] = smem_desc_sw128(smem_u32(S.a[h]));
+            if (wait_phase(&S.a_full, 0, err, status)) {
+                for (int j = 0; j < n_stages; ++j) {
+                    const int slot = j % kNumB, ts = j & 1;
+                    if (!wait_phase(&S.full[slot], (j / kNumB) & 1, err, status)) break;
+                    if (j >= 2 && !wait_phase(&S.tmem_empty[ts], ((j >> 1) - 1) & 1, err, status)) break;
+                    tc_fence_after();
+                    const uint64_t bdesc = smem_desc_sw128(smem_u32(S.b[slot]));
+#pragma unroll
+                    for (int h = 0; h < kIdxHeads; ++h)
+#pragma unroll
+                        for (int k = 0; k < kIdxDim / 16; ++k)
+                            mma_bf16_ss(tmem + ts * 256 + h * kN, adesc[h] + 2 * k, bdesc + 2 * k, idesc, k > 0);
+                    mma_commit(&S.empty[slot]);
+                    mma_commit(&S.tmem_full[ts]);
+                }
+            }
+            // every MMA issued must finish before TMEM is released
+            mma_commit(&S.mma_done);
+            const uint64_t t0 = now_ns();
+            while (!mbar_try_wait(&S.mma_done, 0) && now_ns() - t0 < kWaitNs) {
+            }
+        }
+    } else {
+        // ---------------- epilogue ----------------
+        const int wg = (warp - 2) >> 2;
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const int64_t row_g = row0 + row;
+        const int nc = S.n_c[row];
+        const float w0 = S.w[row][0], w1 = S.w[row][1], w2 = S.w[row][2], w3 = S.w[row][3];
+        const bool live = row_g < n_q && nc > 0;
+        unsigned long long* seg =
+            cand + ((row_g * n_split + split) * 2 + wg) * (int64_t)seg_cap;
+        uint32_t* hist = &S.hist[wg][0][0] + row;  // counter k at hist[k * kM]
+        unsigned theta_key = 0x00800000u;           // key of -FLT_MAX: every finite score passes
+        float theta_f = -FLT_MAX;
+        unsigned cnt = 0, since = 0;
+        int wb = -1;
+        const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + wg * 32;
+
+        for (int j = 0; j < n_stages; ++j) {
+            const int ts = j & 1;
+            if (!wait_phase(&S.tmem_full[ts], (j >> 1) & 1, err, status)) break;
+            tc_fence_after();
+            float a[kIdxHeads][32];
+#pragma unroll
+            for (int h = 0; h < kIdxHeads; ++h) {
+                float lo[16], hi[16];
+                tmem_ld16(tbase + ts * 256 + h * kN, lo);
+                tmem_ld16(tbase + ts * 256 + h * kN + 16, hi);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    a[h][c] = lo[c];
+                    a[h][16 + c] = hi[c];
+                }
+            }
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.tmem_empty[ts]);
+
+            // thresholds published by the other warpgroup (shared memory) and other CTAs (global)
+            {
+                const float other = S.theta[wg ^ 1][row];
+                if ((j & 15) == 15 && live) {
+                    const unsigned g = __ldcg(theta_g + row_g);
+                    if (g > theta_key) theta_key = g;
+                }
+                const unsigned ok = orderable_key(other);
+                if (other > -FLT_MAX && ok > theta_key) theta_key = ok;
+                theta_f = key_to_float(theta_key);
+            }
+            if (!live) continue;
+            const int b_base = blk0 + j * kN + wg * 32;
+            const bool edge = b_base + 32 > nc;
+            float sc[32];
+            unsigned pass = 0;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                float s = w0 * fmaxf(a[0][c], 0.f);
+                s = fmaf(w1, fmaxf(a[1][c], 0.f), s);
+                s = fmaf(w2, fmaxf(a[2][c], 0.f), s);
+                s = fmaf(w3, fmaxf(a[3][c], 0.f), s);
+                if (edge && b_base + c >= nc) s = -INFINITY;
+                sc[c] = s;
+                pass |= (s >= theta_f ? 1u : 0u) << c;
+            }
+            if (pass == 0) continue;
+            // admissions (rare once the threshold has risen): columns in increasing block order
+            float sl[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) sl[c] = sc[c];
+            while (pass) {
+                const int c = __ffs(pass) - 1;
+                pass &= pass - 1;
+                const float s = sl[c];
+                if (!(s >= theta_f)) continue;  // the threshold may have risen within this tile
+                const unsigned key = orderable_key(s);
+                if (cnt < (unsigned)seg_cap) seg[cnt] = ((unsigned long long)key << 32) | (unsigned)(b_base + c);
+                ++cnt;
+                const int bin = (int)(key >> kHistShift);
+                if (wb < 0) wb = max(bin - 56, 0);
+                int jj = bin - wb;
+                if (jj >= kHistBins) {  // keep the window under the largest score seen
+                    const int d = jj - 56;
+                    for (int k = 0; k < kHistBins; ++k) hist[k * kM] = k + d < kHistBins ? hist[(k + d) * kM] : 0;
+                    wb += d;
+                    jj = 56;
+                }
+                if (jj >= 0) hist[jj * kM] += 1;
+                if (++since >= kRaiseEvery) {
+                    since = 0;
+                    unsigned cum = 0;
+                    for (int q = kHistBins - 1; q >= 1; --q) {
+                        cum += hist[q * kM];
+                        if (cum >= (unsigned)kTopK) {
+                            const unsigned edge_key = (unsigned)(wb + q) << kHistShift;
+                            if (edge_key + 1 > theta_key) {
+                                theta_key = edge_key + 1;  // strict for this thread's later blocks
+                                theta_f = key_to_float(theta_key);
+                            }
+                            S.theta[wg][row] = key_to_float(edge_key);
+                            atomicMax(theta_g + row_g, edge_key);
+                            for (int k = 0; k < kHistBins; ++k)
+                                hist[k * kM] = k + q < kHistBins ? hist[(k + q) * kM] : 0;
+                            wb += q;
+                            break;
+                        }
+                    }
+                }
+            }
+        }
+        if (row_g < n_q) cand_cnt[(row_g * n_split + split) * 2 + wg] = cnt;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- finishing select
+
+// One CTA per query row: exact top 512 among the row's admitted blocks (keys at
+// or above the row's final threshold), or every block when n_c <= 512.  Rows whose
+// segments overflowed, or whose survivors do not fit the shared-memory finisher,
+// go to the worklist of k_prefill_fallback.
+__global__ void __launch_bounds__(256)
+k_prefill_finish(const int32_t* __restrict__ q_seq, const int32_t* __restrict__ q_pos, int32_t n_q, int32_t batch,
+                 int64_t kv_capacity, int64_t max_blocks, int n_split, int seg_cap,
+                 const unsigned long long* __restrict__ cand, const unsigned* __restrict__ cand_cnt,
+                 const unsigned* __restrict__ theta_g, int32_t* __restrict__ worklist, int32_t* __restrict__ sel_idx,
+                 int32_t* __restrict__ sel_cnt)
+{
+    __shared__ FinishSmem S;
+    extern __shared__ unsigned long long s_cand[];  // kCandCap entries (dynamic)
+    __shared__ int s_n, s_fail;
+    const int tid = threadIdx.x;
+    const int64_t r = blockIdx.x;
+    const int tile_seq = q_seq[(r / kM) * kM];
+    const int s = q_seq[r], t = q_pos[r];
+    const bool ok = s == tile_seq && s >= 0 && s < batch && t >= 0 && (int64_t)t < kv_capacity;
+    const int64_t n_c = ok ? min(((int64_t)t + 1) / kBlock, max_blocks) : 0;
+    int32_t* out = sel_idx + r * kTopK;
+    if (n_c <= kTopK) {
+        for (int k = tid; k < kTopK; k += 256) out[k] = k < n_c ? k : -1;
+        if (tid == 0) sel_cnt[r] = (int)n_c;
+        return;
+    }
+    const unsigned theta = theta_g[r];
+    if (tid == 0) {
+        s_n = 0;
+        s_fail = 0;
+    }
+    for (int k = tid; k < kTopK; k += 256) S.list[k] = INT_MAX;
+    if (tid == 0) S.n_list = 0;
+    __syncthreads();
+    for (int sg = 0; sg < 2 * n_split; ++sg) {
+        const unsigned c = cand_cnt[r * 2 * n_split + sg];
+        if (c > (unsigned)seg_cap) s_fail = 1;  // overflowed: admitted blocks were dropped
+        const unsigned long long* src = cand + (r * 2 * n_split + sg) * (int64_t)seg_cap;
+        const unsigned cc = min(c, (unsigned)seg_cap);
+        for (unsigned k = tid; k < cc; k += 256) {
+            const unsigned long long e = __ldg(src + k);
+            if ((unsigned)(e >> 32) >= theta) {
+                const int slot = atomicAdd(&s_n, 1);
+                if (slot < kCandCap) s_cand[slot] = e;
+            }
+        }
+    }
+    __syncthreads();
+    const int nc = s_n;
+    if (s_fail || nc > kCandCap || nc < kTopK) {
+        if (tid == 0) worklist[1 + atomicAdd(worklist, 1)] = (int32_t)r;
+        return;
+    }
+    unsigned long long cr[kPerThreadCand];
+#pragma unroll
+    for (int k = 0; k < kPerThreadCand; ++k) {
+        const int j = tid + 256 * k;
+        cr[k] = j < nc ? s_cand[j] : 0ull;
+    }
+    const Cut cut = resolve_cut_regs(S, cr, nc, kTopK, true, 0u);
+    if (!take_by_cut(S, cr, nc, cut)) {
+        if (tid == 0) worklist[1 + atomicAdd(worklist, 1)] = (int32_t)r;
+        return;
+    }
+    bitonic_sort_512(S);
+    for (int k = tid; k < kTopK; k += 256) out[k] = S.list[k];
+    if (tid == 0) sel_cnt[r] = kTopK;
+}
+
+// Rows the streaming pass could not settle: recompute the row's scores with CUDA
+// cores into scratch, then select in block order.  Persistent over the worklist.
+__global__ void __launch_bounds__(256)
+k_prefill_fallback(const __nv_bfloat16* __restrict__ q_idx, const float* __restrict__ w,
+                   const __nv_bfloat16* __restrict__ pooled, const int32_t* __restrict__ q_seq,
+                   const int32_t* __restrict__ q_pos, int64_t kv_capacity, int64_t max_blocks,
+                   const int32_t* __restrict__ worklist, float* __restrict__ scratch, int32_t* __restrict__ sel_idx,
+                   int32_t* __restrict__ sel_cnt)
+{
+    __shared__ FinishSmem S;
+    __shared__ float s_q[kIdxHeads][kIdxDim];
+    const int tid = threadIdx.x;
+    const int n_work = worklist[0];
+    float* row_scores = scratch + (int64_t)blockIdx.x * max_blocks;
+    for (int wi = blockIdx.x; wi < n_work; wi += gridDim.x) {
+        const int64_t r = worklist[1 + wi];
+        const int s = q_seq[r], t = q_pos[r];
+        const int64_t n_c = min(((int64_t)t + 1) / kBlock, max_blocks);
+        __syncthreads();
+        for (int k = tid; k < kIdxHeads * kIdxDim; k += 256)
+            s_q[k / kIdxDim][k % kIdxDim] = __bfloat162float(q_idx[r * kIdxHeads * kIdxDim + k]);
+        __syncthreads();
+        float wv[kIdxHeads];
+#pragma unroll
+        for (int h = 0; h < kIdxHeads; ++h) wv[h] = w[r * kIdxHeads + h];
+        const __nv_bfloat16* prow = pooled + (int64_t)s * (kv_capacity / kBlock) * kIdxDim;
+        for (int64_t b = tid; b < n_c; b += 256) {
+            float acc[kIdxHeads] = {0.f, 0.f, 0.f, 0.f};
+            const uint4* pk = reinterpret_cast<const uint4*>(prow + b * kIdxDim);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 v = __ldg(pk + c);
+                const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float p0 = bf16lo(x[e]), p1 = bf16hi(x[e]);
+#pragma unroll
+                    for (int h = 0; h < kIdxHeads; ++h)
+                        acc[h] = fmaf(s_q[h][8 * c + 2 * e + 1], p1, fmaf(s_q[h][8 * c + 2 * e], p0, acc[h]));
+                }
+            }
+            float sc = 0.f;
+#pragma unroll
+            for (int h = 0; h < kIdxHeads; ++h) sc = fmaf(wv[h], fmaxf(acc[h], 0.f), sc);
+            row_scores[b] = sc;
+        }
+        __threadfence_block();
+        __syncthreads();
+        for (int k = tid; k < kTopK; k += 256) S.list[k] = INT_MAX;
+        __syncthreads();
+        select_by_rescan(S, row_scores, n_c, true, 0u, kTopK);
+        int32_t* out = sel_idx + r * kTopK;
+        const int cnt = (int)min((int64_t)kTopK, n_c);
+        for (int k = tid; k < kTopK; k += 256) out[k] = k < cnt ? S.list[k] : -1;
+        if (tid == 0) sel_cnt[r] = cnt;
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+}  // namespace
+
+int prefill_splits(int32_t n_q, int64_t max_blocks)
+{
+    const int n_tiles = (n_q + kM - 1) / kM;
+    int s = 148 / (n_tiles > 0 ? n_tiles : 1);
+    const int64_t stages = (max_blocks + kN - 1) / kN;
+    const int64_t cap = stages / 4 > 0 ? stages / 4 : 1;  // at least ~4 tiles of work per CTA
+    if (s > cap) s = (int)cap;
+    if (s > 8) s = 8;
+    return s < 1 ? 1 : s;
+}
+
+int prefill_seg_cap() { return 6144; }
+
+size_t prefill_smem_bytes() { return sizeof(K3Smem) + 1024; }
+
+cudaError_t launch_prefill_select(const qsa_dims& d, const void* q_idx, const float* w, const void* pooled,
+                                  const int32_t* q_seq, const int32_t* q_pos, int32_t n_q, int64_t max_blocks,
+                                  int n_split, unsigned long long* cand, unsigned* cand_cnt, unsigned* theta_g,
+                                  int32_t* worklist, float* scratch, int n_fallback_ctas, int32_t* sel_idx,
+                                  int32_t* sel_cnt, unsigned* status, cudaStream_t st)
+{
+    if (n_q <= 0) return cudaSuccess;
+    auto encode = encode_fn();
+    if (!encode) return cudaErrorNotSupported;
+    CUtensorMap tq, tp;
+    {
+        // indexer queries: [n_q][4][64] bf16 as a 3-D tensor (dim, head, query); box = 64 x 1 x 128
+        const cuuint64_t dims[3] = {(cuuint64_t)kIdxDim, (cuuint64_t)kIdxHeads, (cuuint64_t)n_q};
+        const cuuint64_t strides[2] = {(cuuint64_t)kIdxDim * 2, (cuuint64_t)kIdxHeads * kIdxDim * 2};
+        const cuuint32_t box[3] = {(cuuint32_t)kIdxDim, 1u, (cuuint32_t)kM};
+        const cuuint32_t estr[3] = {1u, 1u, 1u};
+        if (encode(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q_idx), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {
+        // pooled keys of all sequences: [B * T/4][64] bf16; box = 64 x 64 blocks
+        const cuuint64_t dims[2] = {(cuuint64_t)kIdxDim, (cuuint64_t)(d.batch * (d.kv_capacity / kBlock))};
+        const cuuint64_t strides[1] = {(cuuint64_t)kIdxDim * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)kIdxDim, (cuuint32_t)kN};
+        const cuuint32_t estr[2] = {1u, 1u};
+        if (encode(&tp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pooled), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    static bool attr_set[128] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const size_t smem = prefill_smem_bytes();
+    if (dev >= 0 && dev < 128 && !attr_set[dev]) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(k_prefill_scores_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    const int seg_cap = prefill_seg_cap();
+    const int n_tiles = (n_q + kM - 1) / kM;
+    k_prefill_scores_tc<<<dim3((unsigned)n_split, (unsigned)n_tiles), kK3Threads, smem, st>>>(
+        tq, tp, w, q_seq, q_pos, n_q, d.batch, d.kv_capacity, max_blocks, n_split, seg_cap, cand, cand_cnt,
+        theta_g, status);
+    static bool fin_attr[128] = {};
+    if (dev >= 0 && dev < 128 && !fin_attr[dev]) {
+        const cudaError_t e = cudaFuncSetAttribute(k_prefill_finish, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)(kCandCap * sizeof(unsigned long long)));
+        if (e != cudaSuccess) return e;
+        fin_attr[dev] = true;
+    }
+    k_prefill_finish<<<(unsigned)n_q, 256, kCandCap * sizeof(unsigned long long), st>>>(q_seq, q_pos, n_q, d.batch, d.kv_capacity, max_blocks, n_split,
+                                                    seg_cap, cand, cand_cnt, theta_g, worklist, sel_idx, sel_cnt);
+    k_prefill_fallback<<<(unsigned)n_fallback_ctas, 256, 0, st>>>(
+        (const __nv_bfloat16*)q_idx, w, (const __nv_bfloat16*)pooled, q_seq, q_pos, d.kv_capacity, max_blocks,
+        worklist, scratch, sel_idx, sel_cnt);
+    return cudaGetLastError();
+}
+
+}  // namespace qsa

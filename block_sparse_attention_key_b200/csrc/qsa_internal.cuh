@@ -79,6 +79,14 @@ struct WsLayout {
     int32_t score_rows = 0;
     size_t sel = 0;        // i32 [n_q][top_k] + i32 [n_q] when the caller passes none
     size_t partial = 0;    // f32 split-K partials
+    // prefill (tensor-core) select
+    size_t pf_cand = 0;    // u64 [n_q][2 * pf_split][seg_cap] admitted (key << 32 | block)
+    size_t pf_cnt = 0;     // u32 [n_q][2 * pf_split]
+    size_t pf_theta = 0;   // u32 [n_q] shared thresholds (zeroed per call)
+    size_t pf_work = 0;    // i32 [1 + n_q] fallback worklist (count zeroed per call)
+    size_t pf_scratch = 0; // f32 [pf_fb_ctas][max_blocks]
+    int pf_split = 0;
+    int pf_fb_ctas = 0;
     size_t total = 0;
     int n_chunks = 0;
     int chunk = 0;
@@ -109,6 +117,16 @@ cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, i
                         int64_t max_blocks, int64_t kv_capacity, int chunk, int n_chunks, TopkCtrl* ctrl,
                         unsigned long long* cand, int32_t* tmp, int32_t* sel_idx, int32_t* sel_cnt, bool hist_done,
                         unsigned* status, cudaStream_t st);
+
+// Prefill chunk (queries of one sequence per 128-row tile): tcgen05 scoring with
+// streaming admission, exact finishing select, fallback for unsettled rows.
+int prefill_splits(int32_t n_q, int64_t max_blocks);
+int prefill_seg_cap();
+cudaError_t launch_prefill_select(const qsa_dims& d, const void* q_idx, const float* w, const void* pooled,
+                                  const int32_t* q_seq, const int32_t* q_pos, int32_t n_q, int64_t max_blocks,
+                                  int n_split, unsigned long long* cand, unsigned* cand_cnt, unsigned* theta_g,
+                                  int32_t* worklist, float* scratch, int n_fallback_ctas, int32_t* sel_idx,
+                                  int32_t* sel_cnt, unsigned* status, cudaStream_t st);
 
 cudaError_t launch_attention(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,
                              const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,

@@ -24,6 +24,7 @@ QSA_DEV_BLOCKS_OVER = 0x4
 QSA_DEV_BAD_LEN = 0x8
 QSA_DEV_BAD_SEL = 0x10
 QSA_DEV_TOO_MANY_NEW = 0x20
+QSA_DEV_TIMEOUT = 0x40
 
 QSA_MODE_DECODE = 0
 QSA_MODE_PREFILL = 1

@@ -75,6 +75,7 @@ extern "C" {
 #define QSA_DEV_BAD_LEN        0x8u  /* len_before/len_after outside [0, kv_capacity] or decreasing */
 #define QSA_DEV_BAD_SEL        0x10u /* sel_idx entry outside [0, n_c(t)) or sel_cnt > top_k: skipped */
 #define QSA_DEV_TOO_MANY_NEW   0x20u /* len_after - len_before > max_new_tokens: rest not pooled */
+#define QSA_DEV_TIMEOUT        0x40u /* a bounded in-kernel wait gave up: results of that call are invalid */
 
 /* ---- forward modes ---- */
 #define QSA_MODE_DECODE  0  /* few queries per sequence: split-K attention, multi-CTA select */

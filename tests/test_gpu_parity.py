@@ -326,3 +326,56 @@ def test_forward_allocates_no_device_memory():
     torch.cuda.synchronize()
     free1, _ = torch.cuda.mem_get_info()
     assert free0 == free1
+
+
+# ------------------------------------------------------------------ prefill (tensor-core select) edge cases
+
+def _prefill_run(wl, q_idx_override=None, q_seq_override=None):
+    import block_sparse_attention_key_b200 as qsa
+    from qsa_synth import device as sdev
+    dw = sdev.DeviceWorkload(wl)
+    gu.pool_history(dw, 0)
+    T = dw.step_tensors(0)
+    if q_idx_override is not None:
+        T["q_idx"] = q_idx_override(T["q_idx"])
+    if q_seq_override is not None:
+        T["q_seq"] = q_seq_override(T["q_seq"])
+    dims = gu.dims_of(wl)
+    n = T["n_q"]
+    ws = gu.new_workspace(qsa.qsa_workspace_bytes(dims, n, T["max_blocks"], qsa.QSA_MODE_PREFILL))
+    out = torch.empty((n, wl.n_q_heads, 128), dtype=torch.bfloat16, device="cuda")
+    sel = torch.empty((n, 512), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((n,), dtype=torch.int32, device="cuda")
+    qsa.qsa_forward(dims, q=T["q"], k_cache=dw.k_cache, v_cache=dw.v_cache, idx_k=dw.idx_k, pooled=dw.pooled,
+                    q_idx=T["q_idx"], w=T["w"], len_before=T["len_before"], len_after=T["len_after"],
+                    q_seq=T["q_seq"], q_pos=T["q_pos"], n_q=n, max_new_tokens=T["max_new_tokens"],
+                    max_blocks=T["max_blocks"], mode=qsa.QSA_MODE_PREFILL, out=out, workspace=ws, sel_idx=sel,
+                    sel_cnt=cnt)
+    return sel.cpu().numpy(), cnt.cpu().numpy(), qsa.qsa_read_device_status(ws)
+
+
+def test_prefill_tie_storm_takes_lowest_blocks():
+    """All indexer queries zero: every score ties at 0, so each row keeps blocks 0..511
+    (this drives the streaming select into its ordered fallback)."""
+    wl = W.Workload("pf_ties", 95, "prefill", 1, 8, 1, 8192, [W._prefill_step(6000, 200)])
+    sel, cnt, flags = _prefill_run(wl, q_idx_override=lambda t: torch.zeros_like(t))
+    assert flags == 0
+    for r in range(200):
+        n_c = (6000 + r + 1) // 4
+        assert cnt[r] == min(512, n_c)
+        np.testing.assert_array_equal(sel[r, : cnt[r]], np.arange(cnt[r]))
+
+
+def test_prefill_row_of_another_sequence_is_rejected():
+    wl = W.Workload("pf_badseq", 94, "prefill", 2, 8, 1, 4096, [W.Step([3000, 0], [3000, 0], [0] * 130,
+                                                                      list(range(2870, 3000)), list(range(130)))])
+
+    def mix(q_seq):
+        q_seq = q_seq.clone()
+        q_seq[5] = 1   # tile 0 belongs to sequence 0
+        return q_seq
+    sel, cnt, flags = _prefill_run(wl, q_seq_override=mix)
+    import block_sparse_attention_key_b200 as qsa
+    assert flags & qsa.qsa.QSA_DEV_BAD_SEQ
+    assert cnt[5] == 0 and (sel[5] == -1).all()
+    assert cnt[4] == 512 and cnt[129] == 512
