@@ -89,9 +89,12 @@ WsLayout plan_workspace(const qsa_dims& d, int32_t n_q, int64_t max_blocks, int3
         off += align_up(segs * prefill_seg_cap() * 8);
         L.pf_cnt = off;
         off += align_up(segs * 4);
-        L.pf_theta = off;                 // thresholds, then the worklist count: zeroed together
+        // thresholds, then the worklist count: zeroed together
+        L.pf_theta = off;
         L.pf_work = off + (size_t)n_q * 4;
         off += align_up((size_t)(2 * n_q + 1) * 4);
+        L.pf_shist = off;
+        off += align_up((size_t)n_q * prefill_shist_words() * 4);
         L.pf_fb_ctas = n_q < 64 ? n_q : 64;
         L.pf_scratch = off;
         off += align_up((size_t)L.pf_fb_ctas * max_blocks * 4);
@@ -275,7 +278,7 @@ int qsa_forward(const qsa_dims* dims, const qsa_forward_args* a, void* workspace
         if (e != cudaSuccess) return QSA_ERR_CUDA;
         e = launch_prefill_select(*dims, a->q_idx, a->w, a->pooled, a->q_seq, a->q_pos, n_q, a->max_blocks,
                                   L.pf_split, (unsigned long long*)(ws + L.pf_cand), (unsigned*)(ws + L.pf_cnt),
-                                  (unsigned*)(ws + L.pf_theta), (int32_t*)(ws + L.pf_work),
+                                  (unsigned*)(ws + L.pf_theta), (uint32_t*)(ws + L.pf_shist), (int32_t*)(ws + L.pf_work),
                                   (float*)(ws + L.pf_scratch), L.pf_fb_ctas, sel_idx, sel_cnt, status, st);
         if (e != cudaSuccess) return QSA_ERR_CUDA;
     } else {

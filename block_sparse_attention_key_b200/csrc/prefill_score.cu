@@ -14,21 +14,24 @@
 //   warp 0      TMA producer: the 4 query tiles once, then 64-block pooled tiles
 //               (8 KiB, 128-byte swizzle) into an 8-deep ring;
 //   warp 1      TMEM allocator and MMA issuer: per pooled tile, 4 heads x 4 K-steps of
-//               tcgen05.mma (M=128, N=64, K=16, bf16 -> f32) into one of two
-//               accumulator stages (4 heads x 64 columns each);
-//   warps 2..9  epilogue, two warpgroups; each thread owns one query row (its TMEM
-//               lane) and half the columns of every tile: tcgen05.ld, ReLU, weights,
-//               head sum, causal cut, and a streaming admission test.
-// Admission: a row keeps every block whose score is at least its threshold.  The
-// threshold starts below every finite score and rises as the row's admitted
-// scores fill a 64-bin histogram (1/16-octave bins of the order-preserving key):
-// once 512 admitted blocks lie at or above a bin edge, no later block below that
-// edge can reach the top 512, and (as blocks arrive in increasing index order) a
-// later block equal to the edge loses every tie, so the thread's own cut is strict.
-// Thresholds are shared (non-strictly) with the other warpgroup through shared
-// memory and with other CTAs of the row through a global atomic max.  Admitted
-// (key, block) pairs are appended to per-(row, CTA, warpgroup) segments in global
-// memory; a finishing kernel selects the exact top 512 among them.
+//               tcgen05.mma (M=128, N=64, K=16, bf16 -> f32) into accumulator stage
+//               (tile & 1), 4 heads x 64 columns each;
+//   warps 2..9  epilogue, two warpgroups: warpgroup g takes the tiles with
+//               (tile & 1) == g, so while one loads TMEM the other computes; each
+//               thread owns one query row (its TMEM lane): tcgen05.ld, ReLU, weights
+//               (packed f32x2 FMAs), head sum, causal cut, streaming admission.
+//
+// Two launches per chunk.  A sampling launch scores every 16th block and only
+// histograms each row's scores (1/16-octave bins of the order-preserving key).
+// The main launch starts each row's admission threshold at the lower edge of the
+// bin holding its 64th-best sampled score (about 1,000 blocks of the row expected
+// above it) and then raises it as admitted scores fill a histogram: once `need`
+// admitted blocks of a thread lie at or above a bin edge, no later block below it
+// can reach the top 512, and (blocks arrive in increasing index order) a later
+// block equal to it loses every tie, so the thread's own cut is strict.  Thresholds
+// are shared, non-strictly, through a global atomic max per row.  The sampled start
+// is only an estimate: the finishing select checks that at least 512 blocks cleared
+// it and sends the row to the exact fallback otherwise.
 //
 // All waits are bounded (a global-timer limit); on a timeout the kernel records
 // QSA_DEV_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
@@ -53,15 +56,18 @@ constexpr int kEpiWarps = 8;
 constexpr int kK3Threads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kHistBins = 64;
-constexpr int kHistShift = 19;          // 1/16-octave bins of the orderable key
+constexpr int kHistShift = 19;          // main pass: 1/16-octave bins of the orderable key
+constexpr int kSampleShift = 19;        // sampling pass: 1/16-octave bins (a 4-octave window)
 constexpr int kRaiseEvery = 32;         // admissions between threshold updates
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any single wait
+constexpr int kSampleStride = 16;
+constexpr int kSampleKth = 64;
+constexpr int kShistWords = kHistBins + 1;   // per (row, warpgroup): window base, then counts
 
 struct __align__(1024) K3Smem {
     __nv_bfloat16 a[kIdxHeads][kM * kIdxDim];   // 4 x 16 KiB
     __nv_bfloat16 b[kNumB][kN * kIdxDim];       // 8 x 8 KiB
-    uint32_t hist[2][kHistBins][kM];            // 64 KiB
-    float theta[2][kM];                         // published (non-strict) thresholds
+    uint32_t hist[2][kHistBins][kM];            // 64 KiB, counter-major per warpgroup
     float w[kM][kIdxHeads];
     int n_c[kM];
     uint64_t full[kNumB], empty[kNumB];
@@ -69,7 +75,7 @@ struct __align__(1024) K3Smem {
     uint64_t a_full, mma_done;
     uint32_t tmem_base;
     int error;
-    int nc_min, nc_max, seq;
+    int nc_max, seq;
 };
 
 __device__ __forceinline__ uint64_t now_ns()
@@ -83,12 +89,16 @@ __device__ __forceinline__ uint64_t now_ns()
 // kWaitNs passes (then sets the flag).  Returns true only if the phase completed.
 __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volatile int* error, unsigned* status)
 {
-    const uint64_t t0 = now_ns();
-    for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;  // fast path: no timer read
+    uint64_t t0 = 0;
+    for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 63u) {
+        if ((i & 255u) == 0u) {
             if (*error) return false;
-            if (now_ns() - t0 > kWaitNs) {
+            const uint64_t t = now_ns();
+            if (t0 == 0) {
+                t0 = t;
+            } else if (t - t0 > kWaitNs) {
                 *error = 1;
                 set_status(status, QSA_DEV_TIMEOUT);
                 return false;
@@ -97,20 +107,74 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volat
     }
 }
 
+// v[c] for a run-time c without local memory: a 5-level tree of selects.
+__device__ __forceinline__ float pick32(const float (&v)[32], int c)
+{
+    float a[16], b[8], d[4], e[2];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a[i] = (c & 16) ? v[i + 16] : v[i];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) b[i] = (c & 8) ? a[i + 8] : a[i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[i] = (c & 4) ? b[i + 4] : b[i];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) e[i] = (c & 2) ? d[i + 2] : d[i];
+    return (c & 1) ? e[1] : e[0];
+}
+
 __device__ __forceinline__ float key_to_float(unsigned k)
 {
     return __uint_as_float((k & 0x80000000u) ? (k ^ 0x80000000u) : ~k);
 }
 
+__device__ __forceinline__ unsigned long long pack2(float lo, float hi)
+{
+    return ((unsigned long long)__float_as_uint(hi) << 32) | __float_as_uint(lo);
+}
+
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b, unsigned long long c)
+{
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 32 scores of one row: sum_h w_h * ReLU(a_h[c]), the same FMA chain as the decode
+// scorer (w0*r0, then + w1*r1, + w2*r2, + w3*r3), two columns per packed f32x2 FMA.
+__device__ __forceinline__ void row_scores32(const float (&a)[kIdxHeads][32], unsigned long long w0,
+                                             unsigned long long w1, unsigned long long w2, unsigned long long w3,
+                                             float (&sc)[32])
+{
+#pragma unroll
+    for (int c = 0; c < 32; c += 2) {
+        unsigned long long s = fma2(w0, pack2(fmaxf(a[0][c], 0.f), fmaxf(a[0][c + 1], 0.f)), 0ull);
+        s = fma2(w1, pack2(fmaxf(a[1][c], 0.f), fmaxf(a[1][c + 1], 0.f)), s);
+        s = fma2(w2, pack2(fmaxf(a[2][c], 0.f), fmaxf(a[2][c + 1], 0.f)), s);
+        s = fma2(w3, pack2(fmaxf(a[3][c], 0.f), fmaxf(a[3][c + 1], 0.f)), s);
+        sc[c] = __uint_as_float((unsigned)s);
+        sc[c + 1] = __uint_as_float((unsigned)(s >> 32));
+    }
+}
+
 }  // namespace
 
+template <bool kSample>
 __global__ void __launch_bounds__(kK3Threads, 1)
 k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_p,
                     const float* __restrict__ w, const int32_t* __restrict__ q_seq,
                     const int32_t* __restrict__ q_pos, int32_t n_q, int32_t batch, int64_t kv_capacity,
-                    int64_t max_blocks, int n_split, int seg_cap, unsigned long long* __restrict__ cand,
-                    unsigned* __restrict__ cand_cnt, unsigned* __restrict__ theta_g, unsigned* status)
+                    int64_t max_blocks, int n_split, int seg_cap, uint32_t* __restrict__ shist,
+                    unsigned long long* __restrict__ cand, unsigned* __restrict__ cand_cnt,
+                    unsigned* __restrict__ theta_g, unsigned* status)
 {
+    constexpr int bstride = kSample ? kSampleStride : 1;
     extern __shared__ uint8_t smem_raw[];
     K3Smem& S = *reinterpret_cast<K3Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -125,12 +189,11 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.tmem_full[i], 1);
-            mbar_init(&S.tmem_empty[i], kEpiWarps);
+            mbar_init(&S.tmem_empty[i], kEpiWarps / 2);
         }
         mbar_init(&S.a_full, 1);
         mbar_init(&S.mma_done, 1);
         S.error = 0;
-        S.nc_min = INT_MAX;
         S.nc_max = 0;
         S.seq = q_seq[row0];
         fence_mbar_init();
@@ -143,11 +206,11 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
         if (r < n_q) {
             const int s = q_seq[r], t = q_pos[r];
             const bool ok = s == S.seq && s >= 0 && s < batch && t >= 0 && (int64_t)t < kv_capacity;
-            if (!ok && split == 0) set_status(status, s != S.seq ? QSA_DEV_BAD_SEQ : QSA_DEV_BAD_POS);
+            if (!ok && split == 0 && !kSample) set_status(status, s != S.seq ? QSA_DEV_BAD_SEQ : QSA_DEV_BAD_POS);
             if (ok) {
                 int64_t c = ((int64_t)t + 1) / kBlock;
                 if (c > max_blocks) {
-                    if (split == 0) set_status(status, QSA_DEV_BLOCKS_OVER);
+                    if (split == 0 && !kSample) set_status(status, QSA_DEV_BLOCKS_OVER);
                     c = max_blocks;
                 }
                 nc = (int)c;
@@ -156,11 +219,7 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
             for (int h = 0; h < kIdxHeads; ++h) S.w[tid][h] = w[r * kIdxHeads + h];
         }
         S.n_c[tid] = nc;
-        S.theta[0][tid] = S.theta[1][tid] = -FLT_MAX;
-        if (r < n_q) {
-            atomicMin(&S.nc_min, nc);
-            atomicMax(&S.nc_max, nc);
-        }
+        if (r < n_q) atomicMax(&S.nc_max, nc);
     }
     if (warp == 1) {
         tmem_alloc(&S.tmem_base, kTmemCols);
@@ -170,15 +229,16 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
     __syncthreads();
     tc_fence_after();
 
-    // this CTA's range of pooled blocks: a 1/n_split share of the tile's longest row
-    const int nc_max = S.nc_max;
+    // this CTA's range of scored positions (every bstride-th block when sampling):
+    // a 1/n_split share of the tile's longest row
+    const int nc_max = (S.nc_max + bstride - 1) / bstride;
     const int chunk = (((nc_max + n_split - 1) / n_split) + kN - 1) / kN * kN;
     const int blk0 = split * chunk;
     const int blk1 = min(blk0 + chunk, nc_max);
     const int n_stages = blk1 > blk0 ? (blk1 - blk0 + kN - 1) / kN : 0;
     const uint32_t tmem = S.tmem_base;
     volatile int* err = &S.error;
-    const int64_t prow0 = (int64_t)S.seq * (kv_capacity / kBlock);
+    const int64_t prow0 = (int64_t)S.seq * (kv_capacity / kBlock) / bstride;
 
     if (warp == 0) {
         if (lane == 0 && n_stages > 0) {
@@ -196,10 +256,12 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
             }
             if (*err) {
                 // drain: every issued tile and the query tiles must land before the CTA exits
-                wait_phase(&S.a_full, 0, err, status);
+                const uint64_t t0 = now_ns();
+                while (!mbar_try_wait(&S.a_full, 0) && now_ns() - t0 < kWaitNs) {
+                }
                 for (int j = max(0, issued - kNumB); j < issued; ++j) {
-                    const uint64_t t0 = now_ns();
-                    while (!mbar_try_wait(&S.full[j % kNumB], (j / kNumB) & 1) && now_ns() - t0 < kWaitNs) {
+                    const uint64_t t1 = now_ns();
+                    while (!mbar_try_wait(&S.full[j % kNumB], (j / kNumB) & 1) && now_ns() - t1 < kWaitNs) {
                     }
                 }
             }
@@ -233,116 +295,180 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
             }
         }
     } else {
-        // ---------------- epilogue ----------------
+        // ---------------- epilogue: warpgroup g takes tiles j with (j & 1) == g ----------------
         const int wg = (warp - 2) >> 2;
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const int64_t row_g = row0 + row;
-        const int nc = S.n_c[row];
-        const float w0 = S.w[row][0], w1 = S.w[row][1], w2 = S.w[row][2], w3 = S.w[row][3];
+        const int nc = (S.n_c[row] + bstride - 1) / bstride;  // scored positions of this row
         const bool live = row_g < n_q && nc > 0;
-        unsigned long long* seg =
-            cand + ((row_g * n_split + split) * 2 + wg) * (int64_t)seg_cap;
+        const float wf0 = S.w[row][0], wf1 = S.w[row][1], wf2 = S.w[row][2], wf3 = S.w[row][3];
+        const unsigned long long w0 = pack2(wf0, wf0), w1 = pack2(wf1, wf1), w2 = pack2(wf2, wf2),
+                                 w3 = pack2(wf3, wf3);
         uint32_t* hist = &S.hist[wg][0][0] + row;  // counter k at hist[k * kM]
-        unsigned theta_key = 0x00800000u;           // key of -FLT_MAX: every finite score passes
-        float theta_f = -FLT_MAX;
+        int wb = -1;                               // histogram window base (absolute bin)
+        unsigned wcount = 0;                       // keys counted in the window
+        const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + wg * 256;
+
+        // ---- main-pass state ----
+        unsigned long long* seg = cand + ((row_g * n_split + split) * 2 + wg) * (int64_t)seg_cap;
+        unsigned theta_key = 0x00800000u;  // key of -FLT_MAX: every finite score passes
         unsigned cnt = 0, since = 0;
-        int wb = -1;
-        const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + wg * 32;
+        if (!kSample && shist && live && S.n_c[row] > 2 * kTopK) {
+            // starting threshold: lower edge of the bin holding the row's kSampleKth-best
+            // sampled score (merge of the two sampling warpgroups' windows)
+            const uint32_t* h0 = shist + (row_g * 2 + 0) * kShistWords;
+            const uint32_t* h1 = shist + (row_g * 2 + 1) * kShistWords;
+            const int b0 = (int)h0[0], b1 = (int)h1[0];
+            const int hi = max(b0, b1) + kHistBins - 1, lo = min(b0, b1);
+            unsigned cum = 0;
+            for (int bin = hi; bin >= lo; --bin) {
+                const int i0 = bin - b0, i1 = bin - b1;
+                cum += (i0 >= 0 && i0 < kHistBins ? h0[1 + i0] : 0u) + (i1 >= 0 && i1 < kHistBins ? h1[1 + i1] : 0u);
+                if (cum >= (unsigned)kSampleKth) {
+                    const unsigned edge = (unsigned)bin << kSampleShift;
+                    if (edge > theta_key) theta_key = edge;
+                    break;
+                }
+            }
+        }
+        float theta_f = key_to_float(theta_key);
 
-        for (int j = 0; j < n_stages; ++j) {
-            const int ts = j & 1;
-            if (!wait_phase(&S.tmem_full[ts], (j >> 1) & 1, err, status)) break;
+        for (int j = wg; j < n_stages; j += 2) {
+            const int k_own = j >> 1;  // this warpgroup's k-th tile
+            if (!wait_phase(&S.tmem_full[wg], k_own & 1, err, status)) break;
             tc_fence_after();
-            float a[kIdxHeads][32];
-#pragma unroll
-            for (int h = 0; h < kIdxHeads; ++h) {
-                float lo[16], hi[16];
-                tmem_ld16(tbase + ts * 256 + h * kN, lo);
-                tmem_ld16(tbase + ts * 256 + h * kN + 16, hi);
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    a[h][c] = lo[c];
-                    a[h][16 + c] = hi[c];
+            if (!kSample && (k_own & 7) == 7 && live) {
+                const unsigned g = __ldcg(theta_g + row_g);
+                if (g > theta_key) {
+                    theta_key = g;
+                    theta_f = key_to_float(theta_key);
                 }
             }
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.tmem_empty[ts]);
-
-            // thresholds published by the other warpgroup (shared memory) and other CTAs (global)
-            {
-                const float other = S.theta[wg ^ 1][row];
-                if ((j & 15) == 15 && live) {
-                    const unsigned g = __ldcg(theta_g + row_g);
-                    if (g > theta_key) theta_key = g;
-                }
-                const unsigned ok = orderable_key(other);
-                if (other > -FLT_MAX && ok > theta_key) theta_key = ok;
-                theta_f = key_to_float(theta_key);
-            }
-            if (!live) continue;
-            const int b_base = blk0 + j * kN + wg * 32;
-            const bool edge = b_base + 32 > nc;
-            float sc[32];
-            unsigned pass = 0;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                float a[kIdxHeads][32];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                float s = w0 * fmaxf(a[0][c], 0.f);
-                s = fmaf(w1, fmaxf(a[1][c], 0.f), s);
-                s = fmaf(w2, fmaxf(a[2][c], 0.f), s);
-                s = fmaf(w3, fmaxf(a[3][c], 0.f), s);
-                if (edge && b_base + c >= nc) s = -INFINITY;
-                sc[c] = s;
-                pass |= (s >= theta_f ? 1u : 0u) << c;
-            }
-            if (pass == 0) continue;
-            // admissions (rare once the threshold has risen): columns in increasing block order
-            float sl[32];
+                for (int h = 0; h < kIdxHeads; ++h) {
+                    float lo[16], hi[16];
+                    tmem_ld16(tbase + h * kN + half * 32, lo);
+                    tmem_ld16(tbase + h * kN + half * 32 + 16, hi);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) sl[c] = sc[c];
-            while (pass) {
-                const int c = __ffs(pass) - 1;
-                pass &= pass - 1;
-                const float s = sl[c];
-                if (!(s >= theta_f)) continue;  // the threshold may have risen within this tile
-                const unsigned key = orderable_key(s);
-                if (cnt < (unsigned)seg_cap) seg[cnt] = ((unsigned long long)key << 32) | (unsigned)(b_base + c);
-                ++cnt;
-                const int bin = (int)(key >> kHistShift);
-                if (wb < 0) wb = max(bin - 56, 0);
-                int jj = bin - wb;
-                if (jj >= kHistBins) {  // keep the window under the largest score seen
-                    const int d = jj - 56;
-                    for (int k = 0; k < kHistBins; ++k) hist[k * kM] = k + d < kHistBins ? hist[(k + d) * kM] : 0;
-                    wb += d;
-                    jj = 56;
+                    for (int c = 0; c < 16; ++c) {
+                        a[h][c] = lo[c];
+                        a[h][16 + c] = hi[c];
+                    }
                 }
-                if (jj >= 0) hist[jj * kM] += 1;
-                if (++since >= kRaiseEvery) {
-                    since = 0;
-                    unsigned cum = 0;
-                    for (int q = kHistBins - 1; q >= 1; --q) {
-                        cum += hist[q * kM];
-                        if (cum >= (unsigned)kTopK) {
+                tmem_ld_wait();
+                if (half == 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.tmem_empty[wg]);
+                }
+                if (!live) continue;
+                float sc[32];
+                row_scores32(a, w0, w1, w2, w3, sc);
+                const int b_base = blk0 + j * kN + half * 32;
+                if (b_base + 32 > nc) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        if (b_base + c >= nc) sc[c] = -INFINITY;
+                }
+                if (kSample) {
+                    // histogram of every sampled score within 4 octaves of the largest seen
+                    float m = sc[0];
+#pragma unroll
+                    for (int c = 1; c < 31; c += 2) m = max3(m, sc[c], sc[c + 1]);
+                    m = fmaxf(m, sc[31]);
+                    if (m == -INFINITY) continue;
+                    if (wb < 0) wb = max((int)(orderable_key(m) >> kSampleShift) - (kHistBins - 4), 0);
+                    const int top = (int)(orderable_key(m) >> kSampleShift);
+                    if (top - wb >= kHistBins) {  // slide the window up under the largest score
+                        const int d = top - wb - (kHistBins - 4);
+                        for (int k = 0; k < kHistBins; ++k) hist[k * kM] = k + d < kHistBins ? hist[(k + d) * kM] : 0u;
+                        wb += d;
+                    }
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const int jj = (int)(orderable_key(sc[c]) >> kSampleShift) - wb;
+                        if (sc[c] != -INFINITY && jj >= 0) hist[jj * kM] += 1;
+                    }
+                    continue;
+                }
+                float m = sc[0];
+#pragma unroll
+                for (int c = 1; c < 31; c += 2) m = max3(m, sc[c], sc[c + 1]);
+                m = fmaxf(m, sc[31]);
+                if (!(m >= theta_f)) continue;
+                unsigned pass = 0;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) pass |= (sc[c] >= theta_f ? 1u : 0u) << c;
+                // admissions: columns in increasing block order
+                while (pass) {
+                    const int c = __ffs(pass) - 1;
+                    pass &= pass - 1;
+                    const float sv = pick32(sc, c);
+                    if (!(sv >= theta_f)) continue;  // the threshold may have risen within this tile
+                    const unsigned key = orderable_key(sv);
+                    if (cnt < (unsigned)seg_cap) seg[cnt] = ((unsigned long long)key << 32) | (unsigned)(b_base + c);
+                    ++cnt;
+                    // the raise histogram only matters once this segment holds many blocks
+                    if (cnt < (unsigned)(kTopK >> 1)) continue;
+                    const int bin = (int)(key >> kHistShift);
+                    if (wb < 0) wb = max(bin - 56, 0);
+                    int jj = bin - wb;
+                    if (jj >= kHistBins) {  // keep the window under the largest score seen
+                        const int d = jj - 56;
+                        unsigned kept = 0;
+                        for (int k = 0; k < kHistBins; ++k) {
+                            const unsigned v = k + d < kHistBins ? hist[(k + d) * kM] : 0u;
+                            hist[k * kM] = v;
+                            kept += v;
+                        }
+                        wcount = kept;
+                        wb += d;
+                        jj = 56;
+                    }
+                    if (jj >= 0) {
+                        hist[jj * kM] += 1;
+                        ++wcount;
+                    }
+                    if (++since >= kRaiseEvery && wcount >= (unsigned)kTopK + kRaiseEvery) {
+                        since = 0;
+                        // largest q with (keys counted in bins >= q) >= top_k, scanning up from the bottom
+                        unsigned above = wcount;
+                        int q = 0;
+                        while (q < kHistBins - 1) {
+                            const unsigned hq = hist[q * kM];
+                            if (above - hq < (unsigned)kTopK) break;
+                            above -= hq;
+                            ++q;
+                        }
+                        if (q >= 1) {
                             const unsigned edge_key = (unsigned)(wb + q) << kHistShift;
                             if (edge_key + 1 > theta_key) {
                                 theta_key = edge_key + 1;  // strict for this thread's later blocks
                                 theta_f = key_to_float(theta_key);
                             }
-                            S.theta[wg][row] = key_to_float(edge_key);
                             atomicMax(theta_g + row_g, edge_key);
                             for (int k = 0; k < kHistBins; ++k)
-                                hist[k * kM] = k + q < kHistBins ? hist[(k + q) * kM] : 0;
+                                hist[k * kM] = k + q < kHistBins ? hist[(k + q) * kM] : 0u;
+                            wcount = above;
                             wb += q;
-                            break;
                         }
                     }
                 }
             }
         }
-        if (row_g < n_q) cand_cnt[(row_g * n_split + split) * 2 + wg] = cnt;
+        if (kSample) {
+            if (row_g < n_q) {
+                uint32_t* out = shist + (row_g * 2 + wg) * kShistWords;
+                out[0] = (uint32_t)max(wb, 0);
+                for (int k = 0; k < kHistBins; ++k) out[1 + k] = wb < 0 ? 0u : hist[k * kM];
+            }
+        } else if (row_g < n_q) {
+            cand_cnt[(row_g * n_split + split) * 2 + wg] = cnt;
+        }
     }
 
     tc_fence_before();
@@ -352,6 +478,44 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
         tmem_dealloc(tmem, kTmemCols);
     }
 }
+
+// Gather a row's admitted entries with key >= th from its 2*n_split segments into
+// s_cand (up to kCandCap); *n gets the count (may exceed kCandCap), *fail is set if
+// a segment overflowed.  Counts are read in parallel, then one flattened pass.
+__device__ __forceinline__ void gather_segments(const unsigned long long* __restrict__ cand,
+                                                const unsigned* __restrict__ cand_cnt, int64_t r, int n_split,
+                                                int seg_cap, unsigned th, unsigned long long* s_cand, int* n,
+                                                int* fail)
+{
+    __shared__ unsigned s_off[2 * 8 + 1];
+    const int tid = threadIdx.x;
+    const int nseg = 2 * n_split;
+    if (tid < nseg) {
+        const unsigned c = cand_cnt[r * nseg + tid];
+        if (c > (unsigned)seg_cap) *fail = 1;
+        s_off[tid + 1] = min(c, (unsigned)seg_cap);
+    }
+    __syncthreads();
+    if (tid == 0) {
+        s_off[0] = 0;
+        for (int sg = 0; sg < nseg; ++sg) s_off[sg + 1] += s_off[sg];
+    }
+    __syncthreads();
+    const unsigned total = s_off[nseg];
+    const int64_t base = r * nseg * (int64_t)seg_cap;
+#pragma unroll 4
+    for (unsigned k = tid; k < total; k += 256) {
+        int sg = 0;
+        while (sg + 1 < nseg && s_off[sg + 1] <= k) ++sg;
+        const unsigned long long e = __ldg(cand + base + (int64_t)sg * seg_cap + (k - s_off[sg]));
+        if ((unsigned)(e >> 32) >= th) {
+            const int slot = atomicAdd(n, 1);
+            if (slot < kCandCap) s_cand[slot] = e;
+        }
+    }
+    __syncthreads();
+}
+
 
 // ---------------------------------------------------------------- finishing select
 
@@ -389,20 +553,7 @@ k_prefill_finish(const int32_t* __restrict__ q_seq, const int32_t* __restrict__ 
     for (int k = tid; k < kTopK; k += 256) S.list[k] = INT_MAX;
     if (tid == 0) S.n_list = 0;
     __syncthreads();
-    for (int sg = 0; sg < 2 * n_split; ++sg) {
-        const unsigned c = cand_cnt[r * 2 * n_split + sg];
-        if (c > (unsigned)seg_cap) s_fail = 1;  // overflowed: admitted blocks were dropped
-        const unsigned long long* src = cand + (r * 2 * n_split + sg) * (int64_t)seg_cap;
-        const unsigned cc = min(c, (unsigned)seg_cap);
-        for (unsigned k = tid; k < cc; k += 256) {
-            const unsigned long long e = __ldg(src + k);
-            if ((unsigned)(e >> 32) >= theta) {
-                const int slot = atomicAdd(&s_n, 1);
-                if (slot < kCandCap) s_cand[slot] = e;
-            }
-        }
-    }
-    __syncthreads();
+    gather_segments(cand, cand_cnt, r, n_split, seg_cap, theta, s_cand, &s_n, &s_fail);
     const int nc = s_n;
     if (s_fail || nc > kCandCap || nc < kTopK) {
         if (tid == 0) worklist[1 + atomicAdd(worklist, 1)] = (int32_t)r;
@@ -499,6 +650,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
+bool set_smem_once(const void* fn, int bytes, bool (&done)[128])
+{
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 128) return false;
+    if (!done[dev]) {
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+        done[dev] = true;
+    }
+    return true;
+}
+
 }  // namespace
 
 int prefill_splits(int32_t n_q, int64_t max_blocks)
@@ -512,20 +675,26 @@ int prefill_splits(int32_t n_q, int64_t max_blocks)
     return s < 1 ? 1 : s;
 }
 
-int prefill_seg_cap() { return 6144; }
+int prefill_seg_cap() { return 2048; }
+int prefill_shist_words() { return 2 * kShistWords; }
 
 size_t prefill_smem_bytes() { return sizeof(K3Smem) + 1024; }
+
+bool prefill_sampled(const qsa_dims& d, int64_t max_blocks)
+{
+    return d.kv_capacity % (kBlock * kSampleStride) == 0 && max_blocks > 2 * kTopK;
+}
 
 cudaError_t launch_prefill_select(const qsa_dims& d, const void* q_idx, const float* w, const void* pooled,
                                   const int32_t* q_seq, const int32_t* q_pos, int32_t n_q, int64_t max_blocks,
                                   int n_split, unsigned long long* cand, unsigned* cand_cnt, unsigned* theta_g,
-                                  int32_t* worklist, float* scratch, int n_fallback_ctas, int32_t* sel_idx,
-                                  int32_t* sel_cnt, unsigned* status, cudaStream_t st)
+                                  uint32_t* shist, int32_t* worklist, float* scratch, int n_fallback_ctas,
+                                  int32_t* sel_idx, int32_t* sel_cnt, unsigned* status, cudaStream_t st)
 {
     if (n_q <= 0) return cudaSuccess;
     auto encode = encode_fn();
     if (!encode) return cudaErrorNotSupported;
-    CUtensorMap tq, tp;
+    CUtensorMap tq, tp, ts;
     {
         // indexer queries: [n_q][4][64] bf16 as a 3-D tensor (dim, head, query); box = 64 x 1 x 128
         const cuuint64_t dims[3] = {(cuuint64_t)kIdxDim, (cuuint64_t)kIdxHeads, (cuuint64_t)n_q};
@@ -537,41 +706,38 @@ cudaError_t launch_prefill_select(const qsa_dims& d, const void* q_idx, const fl
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    {
-        // pooled keys of all sequences: [B * T/4][64] bf16; box = 64 x 64 blocks
-        const cuuint64_t dims[2] = {(cuuint64_t)kIdxDim, (cuuint64_t)(d.batch * (d.kv_capacity / kBlock))};
-        const cuuint64_t strides[1] = {(cuuint64_t)kIdxDim * 2};
+    const bool sampled = prefill_sampled(d, max_blocks);
+    for (int pass = 0; pass < (sampled ? 2 : 1); ++pass) {
+        // pooled keys of all sequences: [B * T/4][64] bf16, box = 64 x 64 blocks; the sampling
+        // view takes every kSampleStride-th block (row pitch kSampleStride x 128 B)
+        const int stride = pass == 0 ? 1 : kSampleStride;
+        const cuuint64_t dims[2] = {(cuuint64_t)kIdxDim, (cuuint64_t)(d.batch * (d.kv_capacity / kBlock) / stride)};
+        const cuuint64_t strides[1] = {(cuuint64_t)kIdxDim * 2 * stride};
         const cuuint32_t box[2] = {(cuuint32_t)kIdxDim, (cuuint32_t)kN};
         const cuuint32_t estr[2] = {1u, 1u};
-        if (encode(&tp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pooled), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        if (encode(pass == 0 ? &tp : &ts, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pooled), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    static bool attr_set[128] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    const size_t smem = prefill_smem_bytes();
-    if (dev >= 0 && dev < 128 && !attr_set[dev]) {
-        const cudaError_t e =
-            cudaFuncSetAttribute(k_prefill_scores_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
+    static bool attr_main[128] = {}, attr_sample[128] = {}, attr_fin[128] = {};
+    const int smem = (int)prefill_smem_bytes();
+    if (!set_smem_once((const void*)k_prefill_scores_tc<false>, smem, attr_main) ||
+        !set_smem_once((const void*)k_prefill_scores_tc<true>, smem, attr_sample) ||
+        !set_smem_once((const void*)k_prefill_finish, (int)(kCandCap * sizeof(unsigned long long)), attr_fin))
+        return cudaErrorInvalidValue;
     const int seg_cap = prefill_seg_cap();
     const int n_tiles = (n_q + kM - 1) / kM;
-    k_prefill_scores_tc<<<dim3((unsigned)n_split, (unsigned)n_tiles), kK3Threads, smem, st>>>(
-        tq, tp, w, q_seq, q_pos, n_q, d.batch, d.kv_capacity, max_blocks, n_split, seg_cap, cand, cand_cnt,
-        theta_g, status);
-    static bool fin_attr[128] = {};
-    if (dev >= 0 && dev < 128 && !fin_attr[dev]) {
-        const cudaError_t e = cudaFuncSetAttribute(k_prefill_finish, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)(kCandCap * sizeof(unsigned long long)));
-        if (e != cudaSuccess) return e;
-        fin_attr[dev] = true;
-    }
-    k_prefill_finish<<<(unsigned)n_q, 256, kCandCap * sizeof(unsigned long long), st>>>(q_seq, q_pos, n_q, d.batch, d.kv_capacity, max_blocks, n_split,
-                                                    seg_cap, cand, cand_cnt, theta_g, worklist, sel_idx, sel_cnt);
+    if (sampled)  // one CTA per query tile: each thread histograms half of its row's samples
+        k_prefill_scores_tc<true><<<dim3(1u, (unsigned)n_tiles), kK3Threads, smem, st>>>(
+            tq, ts, w, q_seq, q_pos, n_q, d.batch, d.kv_capacity, max_blocks, 1, 0, shist, nullptr, nullptr, nullptr,
+            status);
+    k_prefill_scores_tc<false><<<dim3((unsigned)n_split, (unsigned)n_tiles), kK3Threads, smem, st>>>(
+        tq, tp, w, q_seq, q_pos, n_q, d.batch, d.kv_capacity, max_blocks, n_split, seg_cap,
+        sampled ? shist : nullptr, cand, cand_cnt, theta_g, status);
+    k_prefill_finish<<<(unsigned)n_q, 256, kCandCap * sizeof(unsigned long long), st>>>(
+        q_seq, q_pos, n_q, d.batch, d.kv_capacity, max_blocks, n_split, seg_cap, cand, cand_cnt, theta_g, worklist,
+        sel_idx, sel_cnt);
     k_prefill_fallback<<<(unsigned)n_fallback_ctas, 256, 0, st>>>(
         (const __nv_bfloat16*)q_idx, w, (const __nv_bfloat16*)pooled, q_seq, q_pos, d.kv_capacity, max_blocks,
         worklist, scratch, sel_idx, sel_cnt);

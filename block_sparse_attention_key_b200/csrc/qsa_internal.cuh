@@ -84,6 +84,7 @@ struct WsLayout {
     size_t pf_cnt = 0;     // u32 [n_q][2 * pf_split]
     size_t pf_theta = 0;   // u32 [n_q] shared thresholds (zeroed per call)
     size_t pf_work = 0;    // i32 [1 + n_q] fallback worklist (count zeroed per call)
+    size_t pf_shist = 0;   // u32 [n_q][2][65] sampled score histograms
     size_t pf_scratch = 0; // f32 [pf_fb_ctas][max_blocks]
     int pf_split = 0;
     int pf_fb_ctas = 0;
@@ -122,11 +123,13 @@ cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, i
 // streaming admission, exact finishing select, fallback for unsettled rows.
 int prefill_splits(int32_t n_q, int64_t max_blocks);
 int prefill_seg_cap();
+int prefill_shist_words();
+bool prefill_sampled(const qsa_dims& d, int64_t max_blocks);
 cudaError_t launch_prefill_select(const qsa_dims& d, const void* q_idx, const float* w, const void* pooled,
                                   const int32_t* q_seq, const int32_t* q_pos, int32_t n_q, int64_t max_blocks,
                                   int n_split, unsigned long long* cand, unsigned* cand_cnt, unsigned* theta_g,
-                                  int32_t* worklist, float* scratch, int n_fallback_ctas, int32_t* sel_idx,
-                                  int32_t* sel_cnt, unsigned* status, cudaStream_t st);
+                                  uint32_t* shist, int32_t* worklist, float* scratch, int n_fallback_ctas,
+                                  int32_t* sel_idx, int32_t* sel_cnt, unsigned* status, cudaStream_t st);
 
 cudaError_t launch_attention(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,
                              const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,
