@@ -14,8 +14,9 @@
 // a stage each: S = Q K^T and O += P V on mma.sync bf16 tensor cores with fp32
 // accumulation, online softmax in the exp2 domain with quad shuffles for the row
 // max and sum.  The warps' states merge through shared memory.  Decode calls
-// split the block list over CTAs; the last CTA of a (query, KV head) to finish
-// (a completion counter, never a wait) merges the split partials.
+// split the block list over CTAs (one wave of long CTAs); the last CTA of a
+// (query, KV head) to finish (a completion counter, never a wait) merges the
+// split partials in one pass.
 
 #include "qsa_internal.cuh"
 
@@ -334,27 +335,30 @@ k_sparse_attn(const uint4* __restrict__ q, const uint16_t* __restrict__ k_cache,
     if (!s_last) return;
     __threadfence();
     if (row >= G) return;
+    // one pass with a running maximum; the loads of consecutive splits are independent
     const float* base = partial + pair * n_split * pstride;
-    float Mg = -INFINITY;
-#pragma unroll 8
-    for (int sp = 0; sp < n_split; ++sp) Mg = fmaxf(Mg, __ldcg(base + sp * pstride + row));
-    const float Mgu = Mg == -INFINITY ? 0.f : Mg;
-    float Lg = 0.f, og[16];
+    float Mg = -INFINITY, Lg = 0.f, og[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) og[e] = 0.f;
 #pragma unroll 4
     for (int sp = 0; sp < n_split; ++sp) {
         const float* ps = base + sp * pstride;
-        const float f = exp2f(__ldcg(ps + row) - Mgu);
-        Lg += __ldcg(ps + 16 + row) * f;
+        const float ms = __ldcg(ps + row), ls = __ldcg(ps + 16 + row);
+        float4 v[4];
 #pragma unroll
-        for (int e = 0; e < 16; e += 4) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(ps + 32 + row * kHeadDim + d0 + e));
-            og[e] += v.x * f;
-            og[e + 1] += v.y * f;
-            og[e + 2] += v.z * f;
-            og[e + 3] += v.w * f;
+        for (int e = 0; e < 4; ++e) v[e] = __ldcg(reinterpret_cast<const float4*>(ps + 32 + row * kHeadDim + d0) + e);
+        const float mn = fmaxf(Mg, ms);
+        const float mu = mn == -INFINITY ? 0.f : mn;
+        const float fa = exp2f(Mg - mu), fb = exp2f(ms - mu);
+        Lg = Lg * fa + ls * fb;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            og[4 * e] = og[4 * e] * fa + v[e].x * fb;
+            og[4 * e + 1] = og[4 * e + 1] * fa + v[e].y * fb;
+            og[4 * e + 2] = og[4 * e + 2] * fa + v[e].z * fb;
+            og[4 * e + 3] = og[4 * e + 3] * fa + v[e].w * fb;
         }
+        Mg = mn;
     }
     const float inv = Lg > 0.f ? 1.f / Lg : 0.f;
     uint32_t packed[8];
@@ -365,20 +369,19 @@ k_sparse_attn(const uint4* __restrict__ q, const uint16_t* __restrict__ k_cache,
     dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
 }
 
-int attn_blocks_per_split(int32_t n_q, int32_t n_kv_heads)
-{
-    const int64_t pairs = (int64_t)n_q * n_kv_heads;
-    const int64_t tiles_max = (kMaxSplitBlocks + kTileBlocks - 1) / kTileBlocks;  // 33
-    int64_t tps = (pairs * tiles_max + 1183) / 1184;  // aim at ~8 CTAs per SM of work
-    if (tps < 1) tps = 1;
-    if (tps > tiles_max) tps = tiles_max;
-    return (int)(tps * kTileBlocks);
-}
-
 int attn_splits(int32_t n_q, int32_t n_kv_heads)
 {
-    const int bps = attn_blocks_per_split(n_q, n_kv_heads);
-    return (kMaxSplitBlocks + bps - 1) / bps;
+    // Split each (query, KV head) block list so that the whole grid is one wave at two
+    // CTAs per SM (shared memory allows two) on the 148 SMs of a B200: long CTAs keep
+    // three K/V stages in flight instead of paying their set-up and merge per tile.
+    constexpr int64_t kSlots = 2 * 148;
+    const int64_t tiles_max = (kMaxSplitBlocks + kTileBlocks - 1) / kTileBlocks;  // 33
+    const int64_t pairs = (int64_t)n_q * n_kv_heads;
+    int64_t want = pairs > 0 ? kSlots / pairs : 1;
+    if (want < 1) want = 1;
+    if (want > tiles_max) want = tiles_max;
+    const int64_t tiles_per = (tiles_max + want - 1) / want;
+    return (int)((tiles_max + tiles_per - 1) / tiles_per);
 }
 
 cudaError_t launch_attention(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,

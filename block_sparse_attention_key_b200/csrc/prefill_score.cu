@@ -279,10 +279,12 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
                     if (j >= 2 && !wait_phase(&S.tmem_empty[ts], ((j >> 1) - 1) & 1, err, status)) break;
                     tc_fence_after();
                     const uint64_t bdesc = smem_desc_sw128(smem_u32(S.b[slot]));
+                    // K-step outer, head inner: consecutive MMAs write different
+                    // accumulators, so they overlap instead of waiting on each other
 #pragma unroll
-                    for (int h = 0; h < kIdxHeads; ++h)
+                    for (int k = 0; k < kIdxDim / 16; ++k)
 #pragma unroll
-                        for (int k = 0; k < kIdxDim / 16; ++k)
+                        for (int h = 0; h < kIdxHeads; ++h)
                             mma_bf16_ss(tmem + ts * 256 + h * kN, adesc[h] + 2 * k, bdesc + 2 * k, idesc, k > 0);
                     mma_commit(&S.empty[slot]);
                     mma_commit(&S.tmem_full[ts]);

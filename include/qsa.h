@@ -159,8 +159,10 @@ int qsa_sparse_attn(const qsa_dims* dims, const void* q, const void* k_cache, co
  * results as qsa_sparse_attn, without workspace and ws_bytes.
  * Scratch (split-K partials and completion counters) comes from a 16 MiB array
  * built into the library; every GPU that loads the library holds it until the
- * process exits.  A call needing more than that (roughly: more than 128 decode
- * queries with 4 KV heads) returns QSA_ERR_WORKSPACE_TOO_SMALL before launching.
+ * process exits.  A call takes 4 bytes per (query, KV head) pair for counters
+ * plus, when its block lists are split over CTAs (at most 148 pairs), under
+ * 2.5 MiB of partials; one needing more than 16 MiB (more than about 4 million
+ * pairs) returns QSA_ERR_WORKSPACE_TOO_SMALL before launching.
  * The first call on each device, with that device current, looks the array's
  * device address up (cudaGetSymbolAddress); make that first call before any
  * stream capture.  All calls share the array: counters are cleared at the start

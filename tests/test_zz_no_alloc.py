@@ -65,10 +65,10 @@ def test_noalloc_matches_workspace_entry_point_twice(setup):
 def test_noalloc_rejects_calls_beyond_its_scratch(setup):
     qsa, wl, dw, T, sel, cnt = setup
     lib = qsa.load()
-    # 256 decode queries x 4 KV heads need ~17 MiB of split partials: over the 16 MiB limit,
-    # refused on the host before anything is launched
-    dims = gu.dims_of(wl)
+    # 65,535 queries x 128 KV heads need 32 MiB of completion counters (4 bytes per
+    # query and KV head): over the 16 MiB limit, refused on the host before any launch
+    dims = qsa.make_dims(batch=1, n_q_heads=128, n_kv_heads=128, kv_capacity=wl.kv_capacity)
     fake = 1 << 40
-    rc = lib.qsa_sparse_attn_noalloc(ctypes.byref(dims), *([fake] * 7), 256, fake, None)
+    rc = lib.qsa_sparse_attn_noalloc(ctypes.byref(dims), *([fake] * 7), 65535, fake, None)
     assert rc == qsa.QSA_ERR_WORKSPACE_TOO_SMALL
     assert lib.qsa_sparse_attn_noalloc(ctypes.byref(dims), *([None] * 7), 16, None, None) == qsa.QSA_ERR_INVALID_ARG
