@@ -328,6 +328,7 @@ def run_ours(args, wl):
                                                   mb, scores, ld, ws_k)
         run_score()
         run_topk = lambda: qsa.qsa_topk_blocks(dims, scores, ld, T["q_pos"], n_q, mb, sel_k, cnt_k, ws_k)
+        run_topk()  # first launch of its kernels outside the timing (module loading)
         kernels["index_scores_us"] = 1e3 * float(np.mean(timed(run_score, args.steps)))
         kernels["topk_us"] = 1e3 * float(np.mean(timed(run_topk, args.steps)))
     run_attn = lambda: qsa.qsa_sparse_attn(dims, T["q"], dw.k_cache, dw.v_cache, T["q_seq"], T["q_pos"], sel_k,

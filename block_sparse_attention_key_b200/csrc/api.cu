@@ -46,7 +46,9 @@ int select_chunk(int64_t max_blocks, int32_t n_rows)
 {
     if (max_blocks <= 0) return 256;
     const int64_t rows = n_rows > 0 ? n_rows : 1;
-    int64_t c = (max_blocks * rows + 591) / 592;  // ~4 CTAs per SM of work
+    // one wave at two CTAs per SM on the 148 SMs of a B200: each CTA streams a long
+    // run of blocks with its copies in flight instead of paying set-up per short chunk
+    int64_t c = (max_blocks * rows + 295) / 296;
     c = (c + 255) / 256 * 256;
     const int64_t cap = (max_blocks + 255) / 256 * 256;
     if (c > cap) c = cap;
@@ -157,7 +159,7 @@ int qsa_pool_block_keys(const qsa_dims* dims, const void* idx_k, void* pooled, c
     if (workspace && !aligned16(workspace)) return QSA_ERR_INVALID_ARG;
     if (max_new_tokens < 0 || (int64_t)max_new_tokens > dims->kv_capacity) return QSA_ERR_INVALID_ARG;
     if (max_new_tokens == 0) return QSA_OK;
-    return cuda_status(launch_pool(*dims, idx_k, pooled, len_before, len_after, max_new_tokens,
+    return cuda_status(launch_pool(*dims, idx_k, pooled, len_before, len_after, max_new_tokens, nullptr, 0,
                                    (unsigned*)workspace, (cudaStream_t)stream));
 }
 
@@ -176,7 +178,7 @@ int qsa_index_scores(const qsa_dims* dims, const void* q_idx, const float* w, co
     if (ld_scores < max_blocks || ld_scores % 4 != 0) return QSA_ERR_INVALID_ARG;
     const int chunk = select_chunk(max_blocks, n_q);
     return cuda_status(launch_score_decode(*dims, q_idx, w, pooled, q_seq, q_pos, 0, n_q, max_blocks, scores,
-                                           ld_scores, chunk, nullptr, (unsigned*)workspace,
+                                           ld_scores, chunk, nullptr, nullptr, nullptr, (unsigned*)workspace,
                                            (cudaStream_t)stream));
 }
 
@@ -257,23 +259,48 @@ int qsa_forward(const qsa_dims* dims, const qsa_forward_args* a, void* workspace
     char* ws = (char*)workspace;
     unsigned* status = (unsigned*)ws;
     cudaError_t e = cudaSuccess;
+    int32_t* sel_idx = a->sel_idx ? a->sel_idx : (int32_t*)(ws + L.sel);
+    int32_t* sel_cnt = a->sel_cnt ? a->sel_cnt : (int32_t*)(ws + L.sel) + (size_t)n_q * kTopK;
+
+    if (n_q > 0 && a->max_blocks > 0 && a->mode == QSA_MODE_DECODE) {
+        // decode chain, each kernel launched as a programmatic dependent of the one
+        // before: pool (+ clearing of the split counters and select control blocks),
+        // scores with the digit-1 histogram, select, attention
+        e = launch_pool(*dims, a->idx_k, a->pooled, a->len_before, a->len_after, a->max_new_tokens, ws + L.attn_cnt,
+                        L.ctrl_bytes, status, st);
+        if (e != cudaSuccess) return QSA_ERR_CUDA;
+        TopkCtrl* ctrl = (TopkCtrl*)(ws + L.ctrl);
+        float* scores = (float*)(ws + L.scores);
+        // rows of up to 16,384 blocks are selected by the scoring kernel's last CTA per row
+        const bool in_kernel = a->max_blocks <= kScoreFinishMaxBlocks;
+        e = launch_score_decode(*dims, a->q_idx, a->w, a->pooled, a->q_seq, a->q_pos, 0, n_q, a->max_blocks, scores,
+                                L.score_ld, L.chunk, ctrl, in_kernel ? sel_idx : nullptr,
+                                in_kernel ? sel_cnt : nullptr, status, st, true);
+        if (e != cudaSuccess) return QSA_ERR_CUDA;
+        if (!in_kernel) {
+            e = launch_topk(scores, L.score_ld, a->q_pos, 0, n_q, a->max_blocks, dims->kv_capacity, L.chunk,
+                            L.n_chunks, ctrl, (unsigned long long*)(ws + L.cand), (int32_t*)(ws + L.tmp), sel_idx,
+                            sel_cnt, true, status, st, true);
+            if (e != cudaSuccess) return QSA_ERR_CUDA;
+        }
+        return cuda_status(launch_attention(*dims, a->q, a->k_cache, a->v_cache, a->q_seq, a->q_pos, sel_idx,
+                                            sel_cnt, n_q, a->out, L.n_split, (float*)(ws + L.partial),
+                                            (unsigned*)(ws + L.attn_cnt), status, st, true));
+    }
 
     if (a->max_new_tokens > 0) {
-        e = launch_pool(*dims, a->idx_k, a->pooled, a->len_before, a->len_after, a->max_new_tokens, status, st);
+        e = launch_pool(*dims, a->idx_k, a->pooled, a->len_before, a->len_after, a->max_new_tokens, nullptr, 0,
+                        status, st);
         if (e != cudaSuccess) return QSA_ERR_CUDA;
     }
     if (n_q == 0) return QSA_OK;
-
-    int32_t* sel_idx = a->sel_idx ? a->sel_idx : (int32_t*)(ws + L.sel);
-    int32_t* sel_cnt = a->sel_cnt ? a->sel_cnt : (int32_t*)(ws + L.sel) + (size_t)n_q * kTopK;
-    TopkCtrl* ctrl = (TopkCtrl*)(ws + L.ctrl);
-    float* scores = (float*)(ws + L.scores);
 
     if (a->max_blocks == 0) {
         e = cudaMemsetAsync(sel_idx, 0xFF, (size_t)n_q * kTopK * 4, st);
         if (e == cudaSuccess) e = cudaMemsetAsync(sel_cnt, 0, (size_t)n_q * 4, st);
         if (e != cudaSuccess) return QSA_ERR_CUDA;
-    } else if (a->mode == QSA_MODE_PREFILL) {
+    } else {
+        // prefill chunk: tensor-core scoring with streaming admission
         e = cudaMemsetAsync(ws + L.pf_theta, 0, (size_t)(n_q + 1) * 4, st);
         if (e != cudaSuccess) return QSA_ERR_CUDA;
         e = launch_prefill_select(*dims, a->q_idx, a->w, a->pooled, a->q_seq, a->q_pos, n_q, a->max_blocks,
@@ -281,26 +308,8 @@ int qsa_forward(const qsa_dims* dims, const qsa_forward_args* a, void* workspace
                                   (unsigned*)(ws + L.pf_theta), (uint32_t*)(ws + L.pf_shist), (int32_t*)(ws + L.pf_work),
                                   (float*)(ws + L.pf_scratch), L.pf_fb_ctas, sel_idx, sel_cnt, status, st);
         if (e != cudaSuccess) return QSA_ERR_CUDA;
-    } else {
-        // decode: scoring + selection of all rows at once
-        for (int32_t row0 = 0; row0 < n_q; row0 += L.score_rows) {
-            const int32_t n = n_q - row0 < L.score_rows ? n_q - row0 : L.score_rows;
-            if (row0 == 0 && n == n_q)  // one batch: clear split counters and control blocks together
-                e = cudaMemsetAsync(ws + L.attn_cnt, 0, L.ctrl_bytes, st);
-            else
-                e = cudaMemsetAsync(ws + L.ctrl, 0, (size_t)n * sizeof(TopkCtrl), st);
-            if (e != cudaSuccess) return QSA_ERR_CUDA;
-            e = launch_score_decode(*dims, a->q_idx, a->w, a->pooled, a->q_seq, a->q_pos, row0, n, a->max_blocks,
-                                    scores, L.score_ld, L.chunk, ctrl, status, st);
-            if (e != cudaSuccess) return QSA_ERR_CUDA;
-            e = launch_topk(scores, L.score_ld, a->q_pos, row0, n, a->max_blocks, dims->kv_capacity, L.chunk,
-                            L.n_chunks, ctrl, (unsigned long long*)(ws + L.cand), (int32_t*)(ws + L.tmp), sel_idx,
-                            sel_cnt,
-                            true, status, st);
-            if (e != cudaSuccess) return QSA_ERR_CUDA;
-        }
     }
-    if (L.n_split > 1 && !(a->max_blocks > 0 && L.score_rows == n_q)) {
+    if (L.n_split > 1) {
         e = cudaMemsetAsync(ws + L.attn_cnt, 0, (size_t)n_q * dims->n_kv_heads * 4, st);
         if (e != cudaSuccess) return QSA_ERR_CUDA;
     }

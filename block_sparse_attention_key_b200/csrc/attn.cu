@@ -83,6 +83,50 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// Merge the split partials (m, l, o) of one (query, KV head) into its G output
+// rows: one pass with a running maximum; the loads of consecutive splits are
+// independent.  kDims dims per thread: 8 (G <= 8 rows, 16 threads a row) or 16.
+template <int kDims>
+__device__ __forceinline__ void merge_splits(const float* __restrict__ base, int n_split, int G,
+                                             __nv_bfloat16* __restrict__ out_rows)
+{
+    constexpr int kTpr = kHeadDim / kDims;  // threads per row
+    constexpr int64_t pstride = 16 * 2 + 16 * kHeadDim;
+    const int row = threadIdx.x / kTpr, d0 = (threadIdx.x % kTpr) * kDims;
+    if (row >= G) return;
+    float Mg = -INFINITY, Lg = 0.f, og[kDims];
+#pragma unroll
+    for (int e = 0; e < kDims; ++e) og[e] = 0.f;
+#pragma unroll 8
+    for (int sp = 0; sp < n_split; ++sp) {
+        const float* ps = base + sp * pstride;
+        const float ms = __ldcg(ps + row), ls = __ldcg(ps + 16 + row);
+        float4 v[kDims / 4];
+#pragma unroll
+        for (int e = 0; e < kDims / 4; ++e)
+            v[e] = __ldcg(reinterpret_cast<const float4*>(ps + 32 + row * kHeadDim + d0) + e);
+        const float mn = fmaxf(Mg, ms);
+        const float mu = mn == -INFINITY ? 0.f : mn;
+        const float fa = exp2f(Mg - mu), fb = exp2f(ms - mu);
+        Lg = Lg * fa + ls * fb;
+#pragma unroll
+        for (int e = 0; e < kDims / 4; ++e) {
+            og[4 * e] = og[4 * e] * fa + v[e].x * fb;
+            og[4 * e + 1] = og[4 * e + 1] * fa + v[e].y * fb;
+            og[4 * e + 2] = og[4 * e + 2] * fa + v[e].z * fb;
+            og[4 * e + 3] = og[4 * e + 3] * fa + v[e].w * fb;
+        }
+        Mg = mn;
+    }
+    const float inv = Lg > 0.f ? 1.f / Lg : 0.f;
+    uint32_t packed[kDims / 2];
+#pragma unroll
+    for (int e = 0; e < kDims / 2; ++e) packed[e] = pack_bf16(og[2 * e] * inv, og[2 * e + 1] * inv);
+    uint4* dst = reinterpret_cast<uint4*>(out_rows + (int64_t)row * kHeadDim + d0);
+#pragma unroll
+    for (int e = 0; e < kDims / 8; ++e) dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads)
@@ -104,19 +148,30 @@ k_sparse_attn(const uint4* __restrict__ q, const uint16_t* __restrict__ k_cache,
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = n_q_heads / n_kv_heads;
 
+    // before griddep_wait: only the layer call's own inputs (row, position, query)
     const int s = q_seq[i];
     const int t = q_pos[i];
     const bool ok = s >= 0 && s < batch && t >= 0 && (int64_t)t < kv_capacity;
+    const int n_c = ok ? (t + 1) / kBlock : 0;
+    const int n_part = ok ? (t + 1) - kBlock * n_c : 0;  // tokens of the partial block
+    // query heads of this KV group -> rows 0..G-1 of a 16-row tile, rows >= G zero
+    for (int k = tid; k < 16 * 16; k += kThreads) {
+        const int row = k >> 4, ch = k & 15;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (row < G && ok) v = __ldg(q + ((int64_t)i * n_q_heads + g * G + row) * 16 + ch);
+        *reinterpret_cast<uint4*>(smem + kSmemQ + swz(row, ch)) = v;
+    }
+
+    griddep_wait();  // the selection comes from the previous kernel
+    griddep_launch_dependents();
     if (!ok && split == 0 && g == 0 && tid == 0)
         set_status(status, (s < 0 || s >= batch) ? QSA_DEV_BAD_SEQ : QSA_DEV_BAD_POS);
-    const int n_c = ok ? (t + 1) / kBlock : 0;
     int cnt = ok ? sel_cnt[i] : 0;
     const int cnt_max = n_c < kTopK ? n_c : kTopK;
     if (cnt < 0 || cnt > cnt_max) {
         if (split == 0 && g == 0 && tid == 0) set_status(status, QSA_DEV_BAD_SEL);
         cnt = cnt < 0 ? 0 : cnt_max;
     }
-    const int n_part = ok ? (t + 1) - kBlock * n_c : 0;  // tokens of the partial block
     const int n_att = cnt + (n_part > 0 ? 1 : 0);
     const int a0 = split * blocks_per_split;
     const int a1 = min(a0 + blocks_per_split, n_att);
@@ -133,13 +188,6 @@ k_sparse_attn(const uint4* __restrict__ q, const uint16_t* __restrict__ k_cache,
             }
         }
         s_blk[k] = b;
-    }
-    // query heads of this KV group -> rows 0..G-1 of a 16-row tile, rows >= G zero
-    for (int k = tid; k < 16 * 16; k += kThreads) {
-        const int row = k >> 4, ch = k & 15;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (row < G && ok) v = __ldg(q + ((int64_t)i * n_q_heads + g * G + row) * 16 + ch);
-        *reinterpret_cast<uint4*>(smem + kSmemQ + swz(row, ch)) = v;
     }
     __syncthreads();
 
@@ -334,39 +382,8 @@ k_sparse_attn(const uint4* __restrict__ q, const uint16_t* __restrict__ k_cache,
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    if (row >= G) return;
-    // one pass with a running maximum; the loads of consecutive splits are independent
-    const float* base = partial + pair * n_split * pstride;
-    float Mg = -INFINITY, Lg = 0.f, og[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) og[e] = 0.f;
-#pragma unroll 4
-    for (int sp = 0; sp < n_split; ++sp) {
-        const float* ps = base + sp * pstride;
-        const float ms = __ldcg(ps + row), ls = __ldcg(ps + 16 + row);
-        float4 v[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) v[e] = __ldcg(reinterpret_cast<const float4*>(ps + 32 + row * kHeadDim + d0) + e);
-        const float mn = fmaxf(Mg, ms);
-        const float mu = mn == -INFINITY ? 0.f : mn;
-        const float fa = exp2f(Mg - mu), fb = exp2f(ms - mu);
-        Lg = Lg * fa + ls * fb;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            og[4 * e] = og[4 * e] * fa + v[e].x * fb;
-            og[4 * e + 1] = og[4 * e + 1] * fa + v[e].y * fb;
-            og[4 * e + 2] = og[4 * e + 2] * fa + v[e].z * fb;
-            og[4 * e + 3] = og[4 * e + 3] * fa + v[e].w * fb;
-        }
-        Mg = mn;
-    }
-    const float inv = Lg > 0.f ? 1.f / Lg : 0.f;
-    uint32_t packed[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) packed[e] = pack_bf16(og[2 * e] * inv, og[2 * e + 1] * inv);
-    uint4* dst = reinterpret_cast<uint4*>(out + ((int64_t)i * n_q_heads + g * G + row) * kHeadDim + d0);
-    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+    if (G <= 8) merge_splits<8>(partial + pair * n_split * pstride, n_split, G, out + ((int64_t)i * n_q_heads + g * G) * kHeadDim);
+    else merge_splits<16>(partial + pair * n_split * pstride, n_split, G, out + ((int64_t)i * n_q_heads + g * G) * kHeadDim);
 }
 
 int attn_splits(int32_t n_q, int32_t n_kv_heads)
@@ -387,7 +404,7 @@ int attn_splits(int32_t n_q, int32_t n_kv_heads)
 cudaError_t launch_attention(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,
                              const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,
                              const int32_t* sel_cnt, int32_t n_q, void* out, int n_split, float* partial,
-                             unsigned* counters, unsigned* status, cudaStream_t st)
+                             unsigned* counters, unsigned* status, cudaStream_t st, bool pdl)
 {
     if (n_q <= 0) return cudaSuccess;
     const int bps = (kMaxSplitBlocks + n_split - 1) / n_split;
@@ -404,11 +421,10 @@ cudaError_t launch_attention(const qsa_dims& d, const void* q, const void* k_cac
         attr_set[dev] = true;
     }
     dim3 grid((unsigned)n_split, (unsigned)d.n_kv_heads, (unsigned)n_q);
-    k_sparse_attn<<<grid, kThreads, kSmemTotal, st>>>(
-        (const uint4*)q, (const uint16_t*)k_cache, (const uint16_t*)v_cache, q_seq, q_pos, sel_idx, sel_cnt,
-        d.batch, d.n_q_heads, d.n_kv_heads, d.kv_capacity, scale_log2, bps_tiles, n_split,
-        (__nv_bfloat16*)out, partial, counters, status);
-    return cudaGetLastError();
+    return launch_k(k_sparse_attn, grid, dim3(kThreads), kSmemTotal, st, pdl, (const uint4*)q,
+                    (const uint16_t*)k_cache, (const uint16_t*)v_cache, q_seq, q_pos, sel_idx, sel_cnt, d.batch,
+                    d.n_q_heads, d.n_kv_heads, d.kv_capacity, scale_log2, bps_tiles, n_split, (__nv_bfloat16*)out,
+                    partial, counters, status);
 }
 
 }  // namespace qsa

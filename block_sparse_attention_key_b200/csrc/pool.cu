@@ -7,7 +7,9 @@
 // as tokens are appended, so each block is pooled exactly once.
 //
 // HBM-bound and tiny (<= 2,048 blocks x 640 B per call): one thread per
-// (block, 8-dim chunk), four 16-byte loads and one 16-byte store.
+// (block, 8-dim chunk), four 16-byte loads and one 16-byte store.  The same
+// launch clears the layer call's select control blocks and split counters, so
+// the decode chain needs no separate memset.
 
 #include "qsa_internal.cuh"
 
@@ -16,9 +18,16 @@ namespace qsa {
 __global__ void __launch_bounds__(256)
 k_pool_append(const uint4* __restrict__ idx_k, uint4* __restrict__ pooled,
               const int32_t* __restrict__ len_before, const int32_t* __restrict__ len_after,
-              int64_t kv_capacity, int32_t max_new_tokens, int32_t max_new_blocks,
-              unsigned* status)
+              int64_t kv_capacity, int32_t max_new_tokens, int32_t max_new_blocks, int pool_ctas,
+              uint4* __restrict__ zero, int64_t zero_words, unsigned* status)
 {
+    griddep_wait();
+    griddep_launch_dependents();
+    // side job of the CTAs of row 0: clear the caller's control region
+    if (zero && blockIdx.y == 0)
+        for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < zero_words; k += (int64_t)gridDim.x * blockDim.x)
+            zero[k] = make_uint4(0, 0, 0, 0);
+    if ((int)blockIdx.x >= pool_ctas) return;
     const int s = blockIdx.y;
     const int lb = len_before[s];
     const int la = len_after[s];
@@ -63,15 +72,18 @@ k_pool_append(const uint4* __restrict__ idx_k, uint4* __restrict__ pooled,
 }
 
 cudaError_t launch_pool(const qsa_dims& d, const void* idx_k, void* pooled, const int32_t* len_before,
-                        const int32_t* len_after, int32_t max_new_tokens, unsigned* status,
-                        cudaStream_t st)
+                        const int32_t* len_after, int32_t max_new_tokens, void* zero, size_t zero_bytes,
+                        unsigned* status, cudaStream_t st)
 {
-    const int32_t max_new_blocks = max_new_tokens / kBlock + 1;
-    const int64_t threads = (int64_t)max_new_blocks * 8;
-    dim3 grid((unsigned)((threads + 255) / 256), (unsigned)d.batch);
-    k_pool_append<<<grid, 256, 0, st>>>((const uint4*)idx_k, (uint4*)pooled, len_before, len_after,
-                                        d.kv_capacity, max_new_tokens, max_new_blocks, status);
-    return cudaGetLastError();
+    const int32_t max_new_blocks = max_new_tokens > 0 ? max_new_tokens / kBlock + 1 : 0;
+    const int pool_ctas = (int)(((int64_t)max_new_blocks * 8 + 255) / 256);
+    const int64_t zero_words = zero ? (int64_t)(zero_bytes / 16) : 0;
+    const int zero_ctas = (int)((zero_words + 1023) / 1024);  // 4 stores per thread
+    const int ctas = pool_ctas > zero_ctas ? pool_ctas : zero_ctas;
+    if (ctas == 0) return cudaSuccess;
+    return launch_k(k_pool_append, dim3((unsigned)ctas, (unsigned)d.batch), dim3(256), 0, st, false,
+                    (const uint4*)idx_k, (uint4*)pooled, len_before, len_after, d.kv_capacity, max_new_tokens,
+                    max_new_blocks, pool_ctas, (uint4*)zero, zero_words, status);
 }
 
 }  // namespace qsa

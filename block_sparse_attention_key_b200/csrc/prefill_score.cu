@@ -572,7 +572,7 @@ k_prefill_finish(const int32_t* __restrict__ q_seq, const int32_t* __restrict__ 
         if (tid == 0) worklist[1 + atomicAdd(worklist, 1)] = (int32_t)r;
         return;
     }
-    bitonic_sort_512(S);
+    sort_list_512(S);
     for (int k = tid; k < kTopK; k += 256) out[k] = S.list[k];
     if (tid == 0) sel_cnt[r] = kTopK;
 }

@@ -34,8 +34,6 @@ enum SelectMode : int {
 // Per-query control block of the decode select, zeroed before every select.
 struct TopkCtrl {
     unsigned hist1[kBins1];
-    unsigned hist2[kBins2];
-    unsigned hist3[kBins3];
     unsigned done[4];      // CTA completion counters of the passes
     unsigned nsel;         // entries appended to the unordered list
     unsigned prefix;       // resolved high bits of the threshold key
@@ -60,6 +58,32 @@ __device__ __forceinline__ unsigned orderable_key(float f)
 __device__ __forceinline__ void set_status(unsigned* status, unsigned bit)
 {
     if (status) atomicOr(status, bit);
+}
+
+// Programmatic dependent launch.  A kernel launched with launch_k(..., pdl = true)
+// may start while the previous kernel in the stream is still running; before
+// griddep_wait() it may only read inputs that were complete before the layer call
+// began.  Every kernel calls griddep_launch_dependents() only after its own
+// griddep_wait(), so a dependent never overlaps anything older than its direct
+// predecessor.  Without a programmatic dependency both are no-ops.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                            Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 // two bf16 packed in a 32-bit word -> two fp32 (exact)
@@ -101,23 +125,30 @@ int attn_splits(int32_t n_q, int32_t n_kv_heads);
 WsLayout plan_workspace(const qsa_dims& d, int32_t n_q, int64_t max_blocks, int32_t mode);
 
 // ---- launchers (return cudaGetLastError()) ----
+// Pool the blocks completed by the append (max_new_tokens may be 0) and, in the
+// same launch, zero `zero_bytes` (a multiple of 16) at `zero` (may be null).
 cudaError_t launch_pool(const qsa_dims& d, const void* idx_k, void* pooled, const int32_t* len_before,
-                        const int32_t* len_after, int32_t max_new_tokens, unsigned* status,
-                        cudaStream_t st);
+                        const int32_t* len_after, int32_t max_new_tokens, void* zero, size_t zero_bytes,
+                        unsigned* status, cudaStream_t st);
 
-// Scores for rows [row0, row0 + n_rows) (query i = row0 + r, optionally via row_list).
-// With ctrl != nullptr also builds the digit-1 histogram and runs the first select analysis.
+// Scores for rows [row0, row0 + n_rows) (query i = row0 + r).  With ctrl != nullptr
+// also builds the digit-1 histogram; then, with sel_idx != nullptr (needs
+// max_blocks <= 16,384) the last CTA of each row selects the row completely,
+// otherwise it resolves digit 1 for launch_topk.
 cudaError_t launch_score_decode(const qsa_dims& d, const void* q_idx, const float* w, const void* pooled,
                                 const int32_t* q_seq, const int32_t* q_pos, int32_t row0, int32_t n_rows,
                                 int64_t max_blocks, float* scores, int64_t ld, int chunk, TopkCtrl* ctrl,
-                                unsigned* status, cudaStream_t st);
+                                int32_t* sel_idx, int32_t* sel_cnt, unsigned* status, cudaStream_t st,
+                                bool pdl = false);
+// Largest max_blocks for which launch_score_decode can finish the select itself.
+constexpr int64_t kScoreFinishMaxBlocks = 16384;
 
 // Radix select over score rows [0, n_rows) (query i = row0 + r).  If `hist_done`
 // the digit-1 histogram was built by the scoring kernel.
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, int32_t row0, int32_t n_rows,
                         int64_t max_blocks, int64_t kv_capacity, int chunk, int n_chunks, TopkCtrl* ctrl,
                         unsigned long long* cand, int32_t* tmp, int32_t* sel_idx, int32_t* sel_cnt, bool hist_done,
-                        unsigned* status, cudaStream_t st);
+                        unsigned* status, cudaStream_t st, bool pdl = false);
 
 // Prefill chunk (queries of one sequence per 128-row tile): tcgen05 scoring with
 // streaming admission, exact finishing select, fallback for unsettled rows.
@@ -134,6 +165,6 @@ cudaError_t launch_prefill_select(const qsa_dims& d, const void* q_idx, const fl
 cudaError_t launch_attention(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,
                              const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,
                              const int32_t* sel_cnt, int32_t n_q, void* out, int n_split, float* partial,
-                             unsigned* counters, unsigned* status, cudaStream_t st);
+                             unsigned* counters, unsigned* status, cudaStream_t st, bool pdl = false);
 
 }  // namespace qsa

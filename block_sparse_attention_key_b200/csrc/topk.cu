@@ -12,14 +12,17 @@
 // last CTA fixes the boundary bin b1.  One more pass over the row (k_topk_collect)
 // appends every block above b1 to a winner list and every block inside b1 to a
 // candidate list; the CTA that finishes that pass last (a completion counter, no
-// waiting) settles the remaining 20 key bits and the index tie-break among the
-// candidates in registers and shared memory, then bitonic-sorts the 512 winners.
+// waiting) settles the selection among the candidates in shared memory (up to 512
+// candidates: one sort by key descending and block ascending; more: the remaining
+// 20 key bits by radix, then the index tie-break), then sorts the 512 winners.
 // When the boundary bin is too crowded (> 4096 candidates, or > 1024 keys equal
 // at the cut) the finishing CTA instead re-scans the row in index order.
 
 #include "select_finish.cuh"
 
 namespace qsa {
+
+constexpr int kPerThreadLoad = 16;  // score values each collecting thread holds per sub-chunk
 
 // First histogram pass for score rows that come from the caller (qsa_topk_blocks).
 __global__ void __launch_bounds__(256)
@@ -29,6 +32,8 @@ k_topk_pass1(const float* __restrict__ scores, int64_t ld, const int32_t* __rest
     __shared__ unsigned s_hist[kBins1];
     __shared__ unsigned s_warp[8];
     __shared__ int s_last;
+    griddep_wait();
+    griddep_launch_dependents();
     const int tid = threadIdx.x;
     const int r = blockIdx.y;
     TopkCtrl* c = ctrl + r;
@@ -64,6 +69,8 @@ k_topk_collect(const float* __restrict__ scores, int64_t ld, int32_t row0, int c
     __shared__ int s_base[2];
     __shared__ int s_last;
 
+    griddep_wait();  // everything below reads the scoring pass's results
+    griddep_launch_dependents();
     const int tid = threadIdx.x;
     const int r = blockIdx.y;
     const int i = row0 + r;
@@ -78,34 +85,66 @@ k_topk_collect(const float* __restrict__ scores, int64_t ld, int32_t row0, int c
     unsigned long long* cl = cand + (int64_t)r * kCandCap;
 
     if (mode != kSelAll) {
+        // sub-chunks of 256 x kPerThreadLoad blocks: every thread loads its values first
+        // (independent loads), then one block-wide scan places its winners and candidates
         const int64_t b0 = (int64_t)blockIdx.x * chunk;
         const int64_t b_end = min(b0 + (int64_t)chunk, n_c);
-        for (int64_t base = b0; base < b_end; base += 256) {
-            const int64_t b = base + tid;
-            const bool valid = b < b_end;
-            const unsigned key = valid ? orderable_key(__ldg(srow + b)) : 0u;
-            const unsigned top = key >> 20;
-            const bool is_win = valid && (top > b1 || (top == b1 && mode == kSelPrefix));
-            const bool is_cand = valid && top == b1 && mode == kSelUndecided && !crowded;
-            int n_win, n_cand;
-            const int rw = block_rank_256(is_win, S.cnt, &n_win);
-            const int rc = block_rank_256(is_cand, S.cnt, &n_cand);
-            if (n_win == 0 && n_cand == 0) continue;
+        constexpr int kPer = kPerThreadLoad;
+        for (int64_t base = b0; base < b_end; base += 256 * kPer) {
+            unsigned key[kPer];
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                const int64_t b = base + tid + 256 * k;
+                key[k] = b < b_end ? orderable_key(__ldg(srow + b)) : 0u;
+            }
+            unsigned wmask = 0, cmask = 0;
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                const int64_t b = base + tid + 256 * k;
+                const unsigned top = key[k] >> 20;
+                const bool valid = b < b_end;
+                if (valid && (top > b1 || (top == b1 && mode == kSelPrefix))) wmask |= 1u << k;
+                if (valid && top == b1 && mode == kSelUndecided && !crowded) cmask |= 1u << k;
+            }
+            // packed counts: winners in the high 16 bits, candidates in the low 16
+            const unsigned mine = ((unsigned)__popc(wmask) << 16) | (unsigned)__popc(cmask);
+            unsigned incl = mine;
+            const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const unsigned o = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += o;
+            }
+            if (lane == 31) S.warp[warp] = incl;
+            __syncthreads();
+            unsigned before = 0, total = 0;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                const unsigned v = S.warp[w];
+                before += w < warp ? v : 0u;
+                total += v;
+            }
             if (tid == 0) {
-                s_base[0] = n_win ? (int)atomicAdd(&c->nsel, (unsigned)n_win) : 0;
-                s_base[1] = n_cand ? (int)atomicAdd(&c->ncand, (unsigned)n_cand) : 0;
+                s_base[0] = (total >> 16) ? (int)atomicAdd(&c->nsel, total >> 16) : 0;
+                s_base[1] = (total & 0xFFFFu) ? (int)atomicAdd(&c->ncand, total & 0xFFFFu) : 0;
             }
             __syncthreads();
-            if (is_win) {
-                const int slot = s_base[0] + rw;
-                if (slot < kTopK) win[slot] = (int32_t)b;
-                else set_status(status, QSA_DEV_BAD_SEL);
+            const unsigned excl = before + incl - mine;
+            int wslot = s_base[0] + (int)(excl >> 16), cslot = s_base[1] + (int)(excl & 0xFFFFu);
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                const int64_t b = base + tid + 256 * k;
+                if (wmask >> k & 1u) {
+                    if (wslot < kTopK) win[wslot] = (int32_t)b;
+                    else set_status(status, QSA_DEV_BAD_SEL);
+                    ++wslot;
+                }
+                if (cmask >> k & 1u) {
+                    if (cslot < kCandCap) cl[cslot] = ((unsigned long long)key[k] << 32) | (unsigned)b;
+                    ++cslot;
+                }
             }
-            if (is_cand) {
-                const int slot = s_base[1] + rc;
-                if (slot < kCandCap) cl[slot] = ((unsigned long long)key << 32) | (unsigned)b;
-            }
-            __syncthreads();
+            __syncthreads();  // S.warp and s_base are reused by the next sub-chunk
         }
     }
 
@@ -139,20 +178,25 @@ k_topk_collect(const float* __restrict__ scores, int64_t ld, int32_t row0, int c
             const int j = tid + 256 * k;
             cr[k] = j < nc ? __ldcg(cl + j) : 0ull;
         }
-        const Cut cut = resolve_cut_regs(S, cr, nc, need1, false, b1);
         const int n_win = (int)min(__ldcg(&c->nsel), (unsigned)kTopK);
         for (int k = tid; k < n_win; k += 256) S.list[k] = __ldcg(win + k);
         if (tid == 0) S.n_list = n_win;
         __syncthreads();
-        if (!take_by_cut(S, cr, nc, cut)) {
-            for (int k = tid; k < kTopK; k += 256) S.list[k] = INT_MAX;
-            __syncthreads();
-            select_by_rescan(S, srow, n_c, false, b1, need1);
-            sorted = true;
+        if (nc <= kTopK) {
+            // few candidates: sort them by (key desc, block asc) and take the first need1
+            take_top_sorted(S, cr, nc, need1);
+        } else {
+            const Cut cut = resolve_cut_regs(S, cr, nc, need1, false, b1);
+            if (!take_by_cut(S, cr, nc, cut)) {
+                for (int k = tid; k < kTopK; k += 256) S.list[k] = INT_MAX;
+                __syncthreads();
+                select_by_rescan(S, srow, n_c, false, b1, need1);
+                sorted = true;
+            }
         }
     }
     __syncthreads();
-    if (!sorted) bitonic_sort_512(S);
+    if (!sorted) sort_list_512(S);
     int32_t* out = sel_idx + (int64_t)i * kTopK;
     for (int k = tid; k < kTopK; k += 256) out[k] = k < cnt ? S.list[k] : -1;
     if (tid == 0) sel_cnt[i] = cnt;
@@ -161,14 +205,17 @@ k_topk_collect(const float* __restrict__ scores, int64_t ld, int32_t row0, int c
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, int32_t row0, int32_t n_rows,
                         int64_t max_blocks, int64_t kv_capacity, int chunk, int n_chunks, TopkCtrl* ctrl,
                         unsigned long long* cand, int32_t* tmp, int32_t* sel_idx, int32_t* sel_cnt, bool hist_done,
-                        unsigned* status, cudaStream_t st)
+                        unsigned* status, cudaStream_t st, bool pdl)
 {
     if (n_rows <= 0) return cudaSuccess;
     dim3 grid((unsigned)(n_chunks > 0 ? n_chunks : 1), (unsigned)n_rows);
-    if (!hist_done)
-        k_topk_pass1<<<grid, 256, 0, st>>>(scores, ld, q_pos, row0, kv_capacity, max_blocks, chunk, ctrl);
-    k_topk_collect<<<grid, 256, 0, st>>>(scores, ld, row0, chunk, ctrl, cand, tmp, sel_idx, sel_cnt, status);
-    return cudaGetLastError();
+    if (!hist_done) {
+        const cudaError_t e = launch_k(k_topk_pass1, grid, dim3(256), 0, st, false, scores, ld, q_pos, row0,
+                                       kv_capacity, max_blocks, chunk, ctrl);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_k(k_topk_collect, grid, dim3(256), 0, st, hist_done ? pdl : true, scores, ld, row0, chunk, ctrl,
+                    cand, tmp, sel_idx, sel_cnt, status);
 }
 
 }  // namespace qsa

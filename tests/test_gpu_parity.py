@@ -330,9 +330,10 @@ def test_forward_allocates_no_device_memory():
 
 # ------------------------------------------------------------------ prefill (tensor-core select) edge cases
 
-def _prefill_run(wl, q_idx_override=None, q_seq_override=None):
+def _prefill_run(wl, q_idx_override=None, q_seq_override=None, mode=None, return_inputs=False):
     import block_sparse_attention_key_b200 as qsa
     from qsa_synth import device as sdev
+    mode = qsa.QSA_MODE_PREFILL if mode is None else mode
     dw = sdev.DeviceWorkload(wl)
     gu.pool_history(dw, 0)
     T = dw.step_tensors(0)
@@ -342,16 +343,17 @@ def _prefill_run(wl, q_idx_override=None, q_seq_override=None):
         T["q_seq"] = q_seq_override(T["q_seq"])
     dims = gu.dims_of(wl)
     n = T["n_q"]
-    ws = gu.new_workspace(qsa.qsa_workspace_bytes(dims, n, T["max_blocks"], qsa.QSA_MODE_PREFILL))
+    ws = gu.new_workspace(qsa.qsa_workspace_bytes(dims, n, T["max_blocks"], mode))
     out = torch.empty((n, wl.n_q_heads, 128), dtype=torch.bfloat16, device="cuda")
     sel = torch.empty((n, 512), dtype=torch.int32, device="cuda")
     cnt = torch.empty((n,), dtype=torch.int32, device="cuda")
     qsa.qsa_forward(dims, q=T["q"], k_cache=dw.k_cache, v_cache=dw.v_cache, idx_k=dw.idx_k, pooled=dw.pooled,
                     q_idx=T["q_idx"], w=T["w"], len_before=T["len_before"], len_after=T["len_after"],
                     q_seq=T["q_seq"], q_pos=T["q_pos"], n_q=n, max_new_tokens=T["max_new_tokens"],
-                    max_blocks=T["max_blocks"], mode=qsa.QSA_MODE_PREFILL, out=out, workspace=ws, sel_idx=sel,
+                    max_blocks=T["max_blocks"], mode=mode, out=out, workspace=ws, sel_idx=sel,
                     sel_cnt=cnt)
-    return sel.cpu().numpy(), cnt.cpu().numpy(), qsa.qsa_read_device_status(ws)
+    res = (sel.cpu().numpy(), cnt.cpu().numpy(), qsa.qsa_read_device_status(ws))
+    return res + ((dw, T),) if return_inputs else res
 
 
 def test_prefill_tie_storm_takes_lowest_blocks():
@@ -379,3 +381,32 @@ def test_prefill_row_of_another_sequence_is_rejected():
     assert flags & qsa.qsa.QSA_DEV_BAD_SEQ
     assert cnt[5] == 0 and (sel[5] == -1).all()
     assert cnt[4] == 512 and cnt[129] == 512
+
+
+@pytest.mark.parametrize("cap", [8192, 65536, 131072])
+def test_forward_decode_ties_take_lowest_blocks(cap):
+    """Decode rows whose scores tie massively at the cut (the select inside the
+    scoring kernel up to 16,384 blocks, the separate select beyond): all-zero
+    indexer queries keep blocks 0..511; queries with a single nonzero dimension per
+    head leave a handful of distinct scores, and the oracle decides the order."""
+    wl = W.Workload(f"dec_ties_{cap}", 93, "decode", 3, 8, 1, cap, [W._decode_step(3, cap - 1, 0)])
+    n_c = cap // 4
+    sel, cnt, flags = _prefill_run(wl, q_idx_override=lambda t: torch.zeros_like(t), mode=0)
+    assert flags == 0
+    for r in range(3):
+        assert cnt[r] == 512
+        np.testing.assert_array_equal(sel[r], np.arange(512))
+
+    def one_dim(t):
+        z = torch.zeros_like(t)
+        z[:, :, 0] = t[:, :, 0]
+        return z
+    sel, cnt, flags, (dw, T) = _prefill_run(wl, q_idx_override=one_dim, mode=0, return_inputs=True)
+    assert flags == 0
+    q_bits = gu.to_bits(one_dim(T["q_idx"]))
+    w = T["w"].cpu().numpy()
+    for r in range(3):
+        pooled_bits = gu.to_bits(dw.pooled[r, :n_c])
+        want = O.select_top_blocks(O.block_scores(q_bits[r], w[r], pooled_bits))
+        assert cnt[r] == len(want)
+        np.testing.assert_array_equal(sel[r, : cnt[r]], want, err_msg=f"row {r}")
