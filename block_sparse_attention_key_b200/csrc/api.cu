@@ -96,7 +96,7 @@ WsLayout plan_workspace(const qsa_dims& d, int32_t n_q, int64_t max_blocks, int3
         L.pf_work = off + (size_t)n_q * 4;
         off += align_up((size_t)(2 * n_q + 1) * 4);
         L.pf_shist = off;
-        off += align_up((size_t)n_q * prefill_shist_words() * 4);
+        off += align_up((size_t)n_q * prefill_shist_words(L.pf_split) * 4);
         L.pf_fb_ctas = n_q < 64 ? n_q : 64;
         L.pf_scratch = off;
         off += align_up((size_t)L.pf_fb_ctas * max_blocks * 4);

@@ -62,7 +62,8 @@ constexpr int kRaiseEvery = 32;         // admissions between threshold updates
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any single wait
 constexpr int kSampleStride = 16;
 constexpr int kSampleKth = 64;
-constexpr int kShistWords = kHistBins + 1;   // per (row, warpgroup): window base, then counts
+constexpr int kShistWords = kHistBins + 1;   // per (row, CTA, warpgroup): window base, then counts
+constexpr uint32_t kNoWindow = 0xFFFFFFFFu;  // window base of a sampler that saw no score
 
 struct __align__(1024) K3Smem {
     __nv_bfloat16 a[kIdxHeads][kM * kIdxDim];   // 4 x 16 KiB
@@ -318,15 +319,24 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
         unsigned cnt = 0, since = 0;
         if (!kSample && shist && live && S.n_c[row] > 2 * kTopK) {
             // starting threshold: lower edge of the bin holding the row's kSampleKth-best
-            // sampled score (merge of the two sampling warpgroups' windows)
-            const uint32_t* h0 = shist + (row_g * 2 + 0) * kShistWords;
-            const uint32_t* h1 = shist + (row_g * 2 + 1) * kShistWords;
-            const int b0 = (int)h0[0], b1 = (int)h1[0];
-            const int hi = max(b0, b1) + kHistBins - 1, lo = min(b0, b1);
+            // sampled score (merge of the windows of every sampling CTA and warpgroup;
+            // a window that saw no sample has base kNoWindow)
+            const uint32_t* hw = shist + row_g * 2 * n_split * kShistWords;
+            const int nw = 2 * n_split;
+            int lo = INT_MAX, hi = -1;
+            for (int k = 0; k < nw; ++k) {
+                const uint32_t bw = hw[k * kShistWords];
+                if (bw == kNoWindow) continue;
+                lo = min(lo, (int)bw);
+                hi = max(hi, (int)bw + kHistBins - 1);
+            }
             unsigned cum = 0;
-            for (int bin = hi; bin >= lo; --bin) {
-                const int i0 = bin - b0, i1 = bin - b1;
-                cum += (i0 >= 0 && i0 < kHistBins ? h0[1 + i0] : 0u) + (i1 >= 0 && i1 < kHistBins ? h1[1 + i1] : 0u);
+            for (int bin = hi; bin >= lo && bin >= 0; --bin) {
+                for (int k = 0; k < nw; ++k) {
+                    const uint32_t bw = hw[k * kShistWords];
+                    const int i = bin - (int)bw;
+                    if (bw != kNoWindow && i >= 0 && i < kHistBins) cum += hw[k * kShistWords + 1 + i];
+                }
                 if (cum >= (unsigned)kSampleKth) {
                     const unsigned edge = (unsigned)bin << kSampleShift;
                     if (edge > theta_key) theta_key = edge;
@@ -464,8 +474,8 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
         }
         if (kSample) {
             if (row_g < n_q) {
-                uint32_t* out = shist + (row_g * 2 + wg) * kShistWords;
-                out[0] = (uint32_t)max(wb, 0);
+                uint32_t* out = shist + ((row_g * n_split + split) * 2 + wg) * kShistWords;
+                out[0] = wb < 0 ? kNoWindow : (uint32_t)wb;
                 for (int k = 0; k < kHistBins; ++k) out[1 + k] = wb < 0 ? 0u : hist[k * kM];
             }
         } else if (row_g < n_q) {
@@ -678,7 +688,7 @@ int prefill_splits(int32_t n_q, int64_t max_blocks)
 }
 
 int prefill_seg_cap() { return 2048; }
-int prefill_shist_words() { return 2 * kShistWords; }
+int prefill_shist_words(int n_split) { return 2 * n_split * kShistWords; }
 
 size_t prefill_smem_bytes() { return sizeof(K3Smem) + 1024; }
 
@@ -730,10 +740,10 @@ cudaError_t launch_prefill_select(const qsa_dims& d, const void* q_idx, const fl
         return cudaErrorInvalidValue;
     const int seg_cap = prefill_seg_cap();
     const int n_tiles = (n_q + kM - 1) / kM;
-    if (sampled)  // one CTA per query tile: each thread histograms half of its row's samples
-        k_prefill_scores_tc<true><<<dim3(1u, (unsigned)n_tiles), kK3Threads, smem, st>>>(
-            tq, ts, w, q_seq, q_pos, n_q, d.batch, d.kv_capacity, max_blocks, 1, 0, shist, nullptr, nullptr, nullptr,
-            status);
+    if (sampled)  // the main pass's CTA grid: each thread histograms its share of its row's samples
+        k_prefill_scores_tc<true><<<dim3((unsigned)n_split, (unsigned)n_tiles), kK3Threads, smem, st>>>(
+            tq, ts, w, q_seq, q_pos, n_q, d.batch, d.kv_capacity, max_blocks, n_split, 0, shist, nullptr, nullptr,
+            nullptr, status);
     k_prefill_scores_tc<false><<<dim3((unsigned)n_split, (unsigned)n_tiles), kK3Threads, smem, st>>>(
         tq, tp, w, q_seq, q_pos, n_q, d.batch, d.kv_capacity, max_blocks, n_split, seg_cap,
         sampled ? shist : nullptr, cand, cand_cnt, theta_g, status);
