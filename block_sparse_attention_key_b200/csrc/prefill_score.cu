@@ -515,13 +515,25 @@ __device__ __forceinline__ void gather_segments(const unsigned long long* __rest
     __syncthreads();
     const unsigned total = s_off[nseg];
     const int64_t base = r * nseg * (int64_t)seg_cap;
-#pragma unroll 4
-    for (unsigned k = tid; k < total; k += 256) {
-        int sg = 0;
-        while (sg + 1 < nseg && s_off[sg + 1] <= k) ++sg;
-        const unsigned long long e = __ldg(cand + base + (int64_t)sg * seg_cap + (k - s_off[sg]));
-        if ((unsigned)(e >> 32) >= th) {
-            const int slot = atomicAdd(n, 1);
+    const int lane = tid & 31;
+    // one shared-memory atomic per warp and round (ballot + prefix), not one per entry
+    for (unsigned k0 = 0; k0 < total; k0 += 256) {
+        const unsigned k = k0 + tid;
+        unsigned long long e = 0ull;
+        if (k < total) {
+            int sg = 0;
+            while (sg + 1 < nseg && s_off[sg + 1] <= k) ++sg;
+            e = __ldg(cand + base + (int64_t)sg * seg_cap + (k - s_off[sg]));
+        }
+        const bool take = k < total && (unsigned)(e >> 32) >= th;
+        const unsigned m = __ballot_sync(0xffffffffu, take);
+        if (!m) continue;
+        const int leader = __ffs(m) - 1;
+        int slot0 = 0;
+        if (lane == leader) slot0 = atomicAdd(n, __popc(m));
+        slot0 = __shfl_sync(0xffffffffu, slot0, leader);
+        if (take) {
+            const int slot = slot0 + __popc(m & ((1u << lane) - 1u));
             if (slot < kCandCap) s_cand[slot] = e;
         }
     }
