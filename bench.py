@@ -202,6 +202,22 @@ def load_traffic(kernel, workload):
     return rec["bytes_per_launch"]
 
 
+def max_over_ranks(x, world, device):
+    """Largest value of x over the job's ranks (the job's time is its slowest rank's)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world, tokens_per_rank, ms_per_step):
+    """Whole-job throughput: every rank processes its own tokens_per_rank in each step."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 def run_ours(args, wl):
     import torch
     import torch.distributed as dist
@@ -223,12 +239,8 @@ def run_ours(args, wl):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def max_ms(x):
+        return max_over_ranks(x, world, "cuda")
 
     if rank == 0:
         qbuild.build()
@@ -309,9 +321,9 @@ def run_ours(args, wl):
     barrier()
     wall = time.perf_counter() - wall0
     clk = clocks.stop() if clocks else None
-    ms_per_step = max_over_ranks(sum(ms) / len(ms))
-    value = world * n_q_unit / (ms_per_step / 1e3)
-    ms_eager = max_over_ranks(float(np.mean(timed(unit, args.steps))))
+    ms_per_step = max_ms(sum(ms) / len(ms))
+    value = job_tokens_per_s(world, n_q_unit, ms_per_step)
+    ms_eager = max_ms(float(np.mean(timed(unit, args.steps))))
 
     # ---- per-kernel breakdown through the standalone entry points (same inputs) ----
     T = steps[-1]
@@ -403,10 +415,10 @@ def run_ours(args, wl):
         graph_e2e.replay()
         torch.cuda.current_stream().synchronize()
         e2e_ms.append(1e3 * (time.perf_counter() - t0))
-    e2e_ms = max_over_ranks(float(np.mean(e2e_ms)))
+    e2e_ms = max_ms(float(np.mean(e2e_ms)))
     h2d = sum(x[1].numel() for x in e2e_steps)
     d2h = sum(x[6].numel() * x[6].element_size() for x in e2e_steps)
-    e2e = {"value": world * n_q_unit / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+    e2e = {"value": job_tokens_per_s(world, n_q_unit, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
            "timing": "host wall clock around one CUDA-graph replay of: one H2D copy of the step's inputs from "
                      "pinned memory, scatter of the appended K/V/indexer rows, qsa_forward, D2H copy of the "
