@@ -1,7 +1,7 @@
 // Thin inline-PTX wrappers for the sm_100a features the prefill scoring kernel
 // uses: mbarriers, TMA tensor loads, tcgen05 (TMEM allocation, MMA, commit, load).
-// Written from the PTX ISA's instruction descriptions.  Every wait is bounded:
-// it gives up after a fixed number of polls and reports failure to the caller.
+// Written from the PTX ISA's instruction descriptions.  mbar_try_wait polls once;
+// the callers bound every wait with a global-timer limit.
 #pragma once
 
 #include <cuda.h>
@@ -46,15 +46,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
         : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
     return ok != 0;
-}
-
-// Wait for the phase with the given parity to complete; false after `max_polls`
-// unsuccessful polls (each try_wait itself blocks for a bounded, hardware-defined time).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t max_polls)
-{
-    for (uint32_t i = 0; i < max_polls; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
-    return false;
 }
 
 // ---------------------------------------------------------------- TMA
