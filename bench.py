@@ -202,6 +202,22 @@ def load_traffic(kernel, workload):
     return rec["bytes_per_launch"]
 
 
+def forward_launches(wl, prefill, T):
+    """Kernels one qsa_forward call launches (the library's launch plan):
+    decode: pool + control-block clearing, scoring (rows of up to 16,384 blocks are
+    also selected there), the two-pass select for longer rows, attention;
+    prefill: pool when tokens are appended, the sampling launch (when the capacity is
+    a multiple of 64 tokens and rows exceed 1,024 blocks), scoring, finishing select,
+    fallback, attention."""
+    mb = T["max_blocks"]
+    if mb == 0:
+        return (1 if T["max_new_tokens"] > 0 else 0) + 1
+    if not prefill:
+        return 1 + 1 + (1 if mb > 16384 else 0) + 1
+    sampled = wl.kv_capacity % 64 == 0 and mb > 1024
+    return (1 if T["max_new_tokens"] > 0 else 0) + (1 if sampled else 0) + 4
+
+
 def max_over_ranks(x, world, device):
     """Largest value of x over the job's ranks (the job's time is its slowest rank's)."""
     if world == 1:
@@ -425,12 +441,7 @@ def run_ours(args, wl):
                      "output, stream sync"}
 
     flags = qsa.qsa_read_device_status(ws)
-    # our kernels per unit: pool (when tokens are appended), score, select x3, attention
-    launches_per_step = sum((1 if T["max_new_tokens"] > 0 else 0) + 4 + 1 for T in steps)
-    if mode == qsa.QSA_MODE_PREFILL:
-        rows = max(1, min(steps[0]["n_q"], (256 << 20) // (4 * max(1, steps[0]["max_blocks"]))))
-        batches = -(-steps[0]["n_q"] // rows)
-        launches_per_step = (1 if steps[0]["max_new_tokens"] > 0 else 0) + 4 * batches + 1
+    launches_per_step = sum(forward_launches(wl, mode == qsa.QSA_MODE_PREFILL, T) for T in steps)
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded SplitMix64 inputs, see DESIGN.md)",
