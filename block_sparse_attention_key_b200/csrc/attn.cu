@@ -14,9 +14,13 @@
 // a stage each: S = Q K^T and O += P V on mma.sync bf16 tensor cores with fp32
 // accumulation, online softmax in the exp2 domain with quad shuffles for the row
 // max and sum.  The warps' states merge through shared memory.  Decode calls
-// split the block list over CTAs (one wave of long CTAs); the last CTA of a
-// (query, KV head) to finish (a completion counter, never a wait) merges the
-// split partials in one pass.
+// split the block list over up to 8 CTAs (one wave of long CTAs) that form a
+// thread-block cluster: the partials meet in the first CTA's shared memory over
+// distributed shared memory and it merges them.  (The allocation-free entry point
+// keeps the global-memory variant: partials in scratch, the last CTA of a
+// (query, KV head) to finish, found by a completion counter, merges them.)
+
+#include <cooperative_groups.h>
 
 #include "qsa_internal.cuh"
 
@@ -31,6 +35,7 @@ constexpr int kThreads = 128;
 constexpr int kRowBytes = kHeadDim * 2;          // 256 B per token row
 constexpr int kStageBytes = kTileTok * kRowBytes; // 16 KiB of K (or V)
 constexpr int kMaxSplitBlocks = kTopK + 1;        // selected blocks + the partial block
+constexpr int kMaxClusterSplits = 8;              // splits of one (query, KV head): a portable cluster
 
 constexpr int kSmemQ = 0;
 constexpr int kSmemK = kSmemQ + 16 * kRowBytes;
@@ -127,6 +132,43 @@ __device__ __forceinline__ void merge_splits(const float* __restrict__ base, int
     for (int e = 0; e < kDims / 8; ++e) dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
 }
 
+// Merge of up to kMaxClusterSplits partials held in this CTA's shared memory
+// (pm[split][row], pl[split][row], po[split][row][128]), same arithmetic as merge_splits.
+template <int kDims>
+__device__ __forceinline__ void merge_cluster(const float* pm, const float* pl, const float* po, int n_split, int G,
+                                              __nv_bfloat16* __restrict__ out_rows)
+{
+    constexpr int kTpr = kHeadDim / kDims;
+    const int row = threadIdx.x / kTpr, d0 = (threadIdx.x % kTpr) * kDims;
+    if (row >= G) return;
+    float Mg = -INFINITY, Lg = 0.f, og[kDims];
+#pragma unroll
+    for (int e = 0; e < kDims; ++e) og[e] = 0.f;
+    for (int sp = 0; sp < n_split; ++sp) {
+        const float ms = pm[sp * 16 + row], ls = pl[sp * 16 + row];
+        const float mn = fmaxf(Mg, ms);
+        const float mu = mn == -INFINITY ? 0.f : mn;
+        const float fa = exp2f(Mg - mu), fb = exp2f(ms - mu);
+        Lg = Lg * fa + ls * fb;
+#pragma unroll
+        for (int e = 0; e < kDims; e += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(po + (sp * 16 + row) * kHeadDim + d0 + e);
+            og[e] = og[e] * fa + v.x * fb;
+            og[e + 1] = og[e + 1] * fa + v.y * fb;
+            og[e + 2] = og[e + 2] * fa + v.z * fb;
+            og[e + 3] = og[e + 3] * fa + v.w * fb;
+        }
+        Mg = mn;
+    }
+    const float inv = Lg > 0.f ? 1.f / Lg : 0.f;
+    uint32_t packed[kDims / 2];
+#pragma unroll
+    for (int e = 0; e < kDims / 2; ++e) packed[e] = pack_bf16(og[2 * e] * inv, og[2 * e + 1] * inv);
+    uint4* dst = reinterpret_cast<uint4*>(out_rows + (int64_t)row * kHeadDim + d0);
+#pragma unroll
+    for (int e = 0; e < kDims / 8; ++e) dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads)
@@ -134,7 +176,7 @@ k_sparse_attn(const uint4* __restrict__ q, const uint16_t* __restrict__ k_cache,
               const uint16_t* __restrict__ v_cache, const int32_t* __restrict__ q_seq,
               const int32_t* __restrict__ q_pos, const int32_t* __restrict__ sel_idx,
               const int32_t* __restrict__ sel_cnt, int batch, int n_q_heads, int n_kv_heads,
-              int64_t kv_capacity, float scale_log2, int blocks_per_split, int n_split,
+              int64_t kv_capacity, float scale_log2, int blocks_per_split, int n_split, int cluster_merge,
               __nv_bfloat16* __restrict__ out, float* __restrict__ partial, unsigned* __restrict__ counters,
               unsigned* status)
 {
@@ -362,7 +404,38 @@ k_sparse_attn(const uint4* __restrict__ q, const uint16_t* __restrict__ k_cache,
         return;
     }
 
-    // split-K: publish this split's (m, l, o), the last split of (i, g) merges all
+    if (cluster_merge) {
+        // The n_split CTAs of this (query, KV head) form one thread-block cluster: each
+        // writes its (m, l, o) into the shared memory of the cluster's first CTA, which
+        // merges them.  Every thread of every CTA reaches both cluster barriers.
+        namespace cg = cooperative_groups;
+        cg::cluster_group cl = cg::this_cluster();
+        cl.sync();  // every CTA is past its main loop and warp merge: K/V staging is free
+        float* lead = cl.map_shared_rank(reinterpret_cast<float*>(smem + kSmemK), 0);
+        float* pm = lead;                    // [kMaxClusterSplits][16]
+        float* pl = lead + kMaxClusterSplits * 16;
+        float* po = lead + 2 * kMaxClusterSplits * 16;  // [kMaxClusterSplits][16][128]
+        if (row < G) {
+            if ((tid & 7) == 0) {
+                pm[split * 16 + row] = M;
+                pl[split * 16 + row] = L;
+            }
+#pragma unroll
+            for (int e = 0; e < 16; e += 4)
+                *reinterpret_cast<float4*>(po + (split * 16 + row) * kHeadDim + d0 + e) =
+                    make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+        }
+        cl.sync();  // all partials are in the first CTA's shared memory
+        if (split != 0) return;
+        const float* lm = reinterpret_cast<const float*>(smem + kSmemK);
+        __nv_bfloat16* orow = out + ((int64_t)i * n_q_heads + g * G) * kHeadDim;
+        if (G <= 8) merge_cluster<8>(lm, lm + kMaxClusterSplits * 16, lm + 2 * kMaxClusterSplits * 16, n_split, G, orow);
+        else merge_cluster<16>(lm, lm + kMaxClusterSplits * 16, lm + 2 * kMaxClusterSplits * 16, n_split, G, orow);
+        return;
+    }
+
+    // split-K through global memory: publish this split's (m, l, o), the last split of
+    // (i, g) merges all
     const int64_t pair = (int64_t)i * n_kv_heads + g;
     const int64_t pstride = 16 * 2 + 16 * kHeadDim;
     float* pp = partial + (pair * n_split + split) * pstride;
@@ -396,7 +469,7 @@ int attn_splits(int32_t n_q, int32_t n_kv_heads)
     const int64_t pairs = (int64_t)n_q * n_kv_heads;
     int64_t want = pairs > 0 ? kSlots / pairs : 1;
     if (want < 1) want = 1;
-    if (want > tiles_max) want = tiles_max;
+    if (want > kMaxClusterSplits) want = kMaxClusterSplits;  // the splits of a pair form one cluster
     const int64_t tiles_per = (tiles_max + want - 1) / want;
     return (int)((tiles_max + tiles_per - 1) / tiles_per);
 }
@@ -404,9 +477,10 @@ int attn_splits(int32_t n_q, int32_t n_kv_heads)
 cudaError_t launch_attention(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,
                              const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,
                              const int32_t* sel_cnt, int32_t n_q, void* out, int n_split, float* partial,
-                             unsigned* counters, unsigned* status, cudaStream_t st, bool pdl)
+                             unsigned* counters, unsigned* status, cudaStream_t st, bool pdl, bool cluster_merge)
 {
     if (n_q <= 0) return cudaSuccess;
+    if (n_split > kMaxClusterSplits) return cudaErrorInvalidValue;
     const int bps = (kMaxSplitBlocks + n_split - 1) / n_split;
     const int bps_tiles = ((bps + kTileBlocks - 1) / kTileBlocks) * kTileBlocks;
     const float scale = d.softmax_scale > 0.f ? d.softmax_scale : 1.0f / sqrtf((float)d.head_dim);
@@ -420,11 +494,32 @@ cudaError_t launch_attention(const qsa_dims& d, const void* q, const void* k_cac
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    dim3 grid((unsigned)n_split, (unsigned)d.n_kv_heads, (unsigned)n_q);
-    return launch_k(k_sparse_attn, grid, dim3(kThreads), kSmemTotal, st, pdl, (const uint4*)q,
-                    (const uint16_t*)k_cache, (const uint16_t*)v_cache, q_seq, q_pos, sel_idx, sel_cnt, d.batch,
-                    d.n_q_heads, d.n_kv_heads, d.kv_capacity, scale_log2, bps_tiles, n_split, (__nv_bfloat16*)out,
-                    partial, counters, status);
+    const bool clustered = cluster_merge && n_split > 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)n_split, (unsigned)d.n_kv_heads, (unsigned)n_q);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemTotal;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (clustered) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)n_split;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.attrs = na ? attr : nullptr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, k_sparse_attn, (const uint4*)q, (const uint16_t*)k_cache,
+                              (const uint16_t*)v_cache, q_seq, q_pos, sel_idx, sel_cnt, d.batch, d.n_q_heads,
+                              d.n_kv_heads, d.kv_capacity, scale_log2, bps_tiles, n_split, clustered ? 1 : 0,
+                              (__nv_bfloat16*)out, partial, counters, status);
 }
 
 }  // namespace qsa

@@ -105,6 +105,6 @@ extern "C" int qsa_sparse_attn_noalloc(const qsa_dims* dims, const void* q, cons
         return QSA_ERR_CUDA;
     // no status word in this variant: out-of-range indices are still skipped, just not reported
     const cudaError_t e = launch_attention(*dims, q, k_cache, v_cache, q_seq, q_pos, sel_idx, sel_cnt, n_q, out,
-                                           n_split, partial, counters, nullptr, st);
+                                           n_split, partial, counters, nullptr, st, false, false);
     return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
 }

@@ -165,6 +165,7 @@ cudaError_t launch_prefill_select(const qsa_dims& d, const void* q_idx, const fl
 cudaError_t launch_attention(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,
                              const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,
                              const int32_t* sel_cnt, int32_t n_q, void* out, int n_split, float* partial,
-                             unsigned* counters, unsigned* status, cudaStream_t st, bool pdl = false);
+                             unsigned* counters, unsigned* status, cudaStream_t st, bool pdl = false,
+                             bool cluster_merge = true);
 
 }  // namespace qsa
