@@ -135,3 +135,24 @@ def test_binding_refuses_cpu_tensors(qsa):
     import torch
     with pytest.raises(ValueError):
         qsa._ptr(torch.zeros(4))
+
+
+def test_binding_constants_match_the_header(qsa):
+    """Every QSA_* value the header defines has the same value in the binding."""
+    text = open(os.path.join(ROOT, "include", "qsa.h")).read()
+    defs = dict(re.findall(r"^#define\s+(QSA_(?:OK|ERR_\w+|DEV_\w+|MODE_\w+))\s+(-?(?:0x)?[0-9A-Fa-f]+)u?\b", text, re.M))
+    assert len(defs) == 14  # 5 return codes, 7 device status bits, 2 modes
+    for name, val in defs.items():
+        assert getattr(qsa, name) == int(val, 0), name
+
+
+def test_workspace_grows_with_queries_and_blocks(qsa):
+    """Workspace is monotone in the query count and the block bound, in both modes."""
+    d = _dims(qsa, batch=4, kv_capacity=1 << 20)
+    for mode in (qsa.QSA_MODE_DECODE, qsa.QSA_MODE_PREFILL):
+        prev = 0
+        for n_q in (1, 16, 256, 4096):
+            w = qsa.qsa_workspace_bytes(d, n_q, 1 << 16, mode)
+            assert w >= prev > 0 or prev == 0
+            prev = w
+        assert qsa.qsa_workspace_bytes(d, 256, 1 << 12, mode) <= qsa.qsa_workspace_bytes(d, 256, 1 << 16, mode)
