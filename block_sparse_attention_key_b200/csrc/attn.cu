@@ -20,6 +20,8 @@
 // keeps the global-memory variant: partials in scratch, the last CTA of a
 // (query, KV head) to finish, found by a completion counter, merges them.)
 
+#include <atomic>
+
 #include <cooperative_groups.h>
 
 #include "qsa_internal.cuh"
@@ -485,14 +487,14 @@ cudaError_t launch_attention(const qsa_dims& d, const void* q, const void* k_cac
     const int bps_tiles = ((bps + kTileBlocks - 1) / kTileBlocks) * kTileBlocks;
     const float scale = d.softmax_scale > 0.f ? d.softmax_scale : 1.0f / sqrtf((float)d.head_dim);
     const float scale_log2 = scale * 1.4426950408889634f;
-    static bool attr_set[128] = {};
+    static std::atomic<bool> attr_set[128];  // per device; setting it twice is harmless
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 128 && !attr_set[dev]) {
+    if (dev >= 0 && dev < 128 && !attr_set[dev].load()) {
         const cudaError_t e =
             cudaFuncSetAttribute(k_sparse_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
         if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+        attr_set[dev].store(true);
     }
     const bool clustered = cluster_merge && n_split > 1;
     cudaLaunchConfig_t cfg = {};

@@ -36,7 +36,9 @@
 // All waits are bounded (a global-timer limit); on a timeout the kernel records
 // QSA_DEV_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
 
+#include <atomic>
 #include <cfloat>
+#include <mutex>
 
 #include <cudaTypedefs.h>
 
@@ -663,25 +665,26 @@ namespace {
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 {
+    static std::once_flag once;
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
+    std::call_once(once, [] {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
             fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
+    });
     return fn;
 }
 
-bool set_smem_once(const void* fn, int bytes, bool (&done)[128])
+bool set_smem_once(const void* fn, int bytes, std::atomic<bool> (&done)[128])
 {
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 128) return false;
-    if (!done[dev]) {
+    if (!done[dev].load()) {  // setting it twice (two host threads) is harmless
         if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
-        done[dev] = true;
+        done[dev].store(true);
     }
     return true;
 }
@@ -744,7 +747,7 @@ cudaError_t launch_prefill_select(const qsa_dims& d, const void* q_idx, const fl
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    static bool attr_main[128] = {}, attr_sample[128] = {}, attr_fin[128] = {};
+    static std::atomic<bool> attr_main[128], attr_sample[128], attr_fin[128];
     const int smem = (int)prefill_smem_bytes();
     if (!set_smem_once((const void*)k_prefill_scores_tc<false>, smem, attr_main) ||
         !set_smem_once((const void*)k_prefill_scores_tc<true>, smem, attr_sample) ||

@@ -20,6 +20,8 @@
 // products is exact for small integers.  Optionally the same pass histograms the
 // scores' top key digit for the select.
 
+#include <atomic>
+
 #include "select_finish.cuh"
 
 namespace qsa {
@@ -214,17 +216,17 @@ cudaError_t launch_score_decode(const qsa_dims& d, const void* q_idx, const floa
     if (n_rows <= 0 || max_blocks <= 0) return cudaSuccess;
     const int64_t n_chunks = (max_blocks + chunk - 1) / chunk;
     dim3 grid((unsigned)n_chunks, (unsigned)n_rows);
-    static bool attr_set[128] = {};
+    static std::atomic<bool> attr_set[128];  // per device; setting it twice is harmless
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 128 && !attr_set[dev]) {
+    if (dev >= 0 && dev < 128 && !attr_set[dev].load()) {
         cudaError_t e = cudaFuncSetAttribute(k_score_decode<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kStageBytes);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(k_score_decode<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      kStageBytes);
         if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+        attr_set[dev].store(true);
     }
     return launch_k(ctrl ? k_score_decode<true> : k_score_decode<false>, grid, dim3(256), kStageBytes, st, pdl,
                     (const uint4*)q_idx, w, (const uint4*)pooled, q_seq, q_pos, row0, d.batch, d.kv_capacity,
