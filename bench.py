@@ -17,6 +17,7 @@ import argparse
 import json
 import os
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -139,7 +140,8 @@ class Clocks:
     """nvidia-smi samples during the timed region."""
 
     def __init__(self, index):
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        out_dir = os.environ.get("QSA_BENCH_OUT") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"clocks_bench_{os.getpid()}.csv")
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -444,7 +446,7 @@ def run_ours(args, wl):
     launches_per_step = sum(forward_launches(wl, mode == qsa.QSA_MODE_PREFILL, T) for T in steps)
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded SplitMix64 inputs, see DESIGN.md)",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded SplitMix64 inputs, integer indexer inputs, approx. N(0,1) Q/K/V)",
             "config": dict(workload_config(wl), parallelism=f"replicas x{world} (independent sequences per GPU)",
                            execution="CUDA graph of the unit's qsa_forward calls"),
             "roofline": roofline, "kernels": kernels, "e2e": e2e,
