@@ -247,6 +247,17 @@ def test_forward_decode_short_and_ragged_positions():
     _forward_vs_oracle(wl)
 
 
+def test_forward_decode_mixed_lengths_two_pass_select():
+    """Rows from a few blocks to 32,768 blocks in one decode call: the host bound exceeds
+    16,384 blocks, so every row goes through the two-pass select (short rows take all
+    their blocks), and the attention splits merge inside clusters."""
+    pos = [100, 2100, 70000, 131071]
+    n = len(pos)
+    wl = W.Workload("mixed_decode", 92, "decode", n, 8, 2, 131072,
+                    [W.Step([p for p in pos], [p + 1 for p in pos], list(range(n)), pos, list(range(n)))])
+    _forward_vs_oracle(wl)
+
+
 def test_forward_decode_two_steps_block_completion():
     # step 1 leaves a 3-token partial block, step 2 completes it (it becomes a candidate)
     cap = 16384
