@@ -14,6 +14,11 @@ constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA; }
+
+}  // namespace
+
+// Argument checks shared by every entry point (declared in qsa_internal.cuh).
 bool aligned16(const void* p) { return p != nullptr && ((uintptr_t)p & 15u) == 0; }
 
 int check_dims(const qsa_dims* d)
@@ -37,10 +42,6 @@ int check_rows(const qsa_dims* d, int32_t n_q, int64_t max_blocks)
     if (n_q > 65535) return QSA_ERR_UNSUPPORTED;
     return QSA_OK;
 }
-
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA; }
-
-}  // namespace
 
 int select_chunk(int64_t max_blocks, int32_t n_rows)
 {

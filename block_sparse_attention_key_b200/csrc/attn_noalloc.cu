@@ -12,14 +12,14 @@
 // loads this library holds that much memory until the process exits.  On the
 // host the array's name is only a stand-in, not a device address, so the first
 // call on each device (with that device current) looks the address up with
-// cudaGetSymbolAddress and caches it; that first call should therefore come
-// before any stream capture.  All calls share the one array and it keeps the
-// previous call's contents: the completion counters are cleared at the start of
+// cudaGetSymbolAddress, and every later call made outside stream capture looks
+// it up again; the first call on each device should therefore come before any
+// stream capture.  All calls share the one array and it keeps the previous
+// call's contents: the completion counters are cleared at the start of
 // every call, and calls whose executions overlap on the GPU (for example on two
 // streams) race on it.  Nothing here calls cudaMalloc, cudaFree or any other
 // allocating routine.
 
-#include <cmath>
 #include <mutex>
 
 #include "qsa_internal.cuh"
@@ -37,37 +37,31 @@ __device__ __align__(256) unsigned char g_attn_scratch[kScratchBytes];
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of g_attn_scratch on the current device (looked up once per device).
-cudaError_t scratch_address(void** out)
+// Device address of g_attn_scratch on the current device.  Looked up afresh on
+// every call made outside stream capture (so a device reset, which rebuilds the
+// context and may move the array, never leaves a stale address in use); a call
+// made while `st` is capturing reuses the address of the last uncaptured call on
+// this device, and fails if there was none.
+cudaError_t scratch_address(cudaStream_t st, void** out)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(st, &cap);
+    if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
+    if (cap == cudaStreamCaptureStatusNone) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_attn_scratch);
         if (e != cudaSuccess) return e;
         g_scratch_ptr[dev] = p;
+    } else if (!g_scratch_ptr[dev]) {
+        return cudaErrorStreamCaptureUnsupported;
     }
     *out = g_scratch_ptr[dev];
     return cudaSuccess;
-}
-
-bool aligned16(const void* p) { return p != nullptr && ((uintptr_t)p & 15u) == 0; }
-
-int check_args(const qsa_dims* d, int32_t n_q)
-{
-    if (!d || d->batch < 1 || d->n_q_heads < 1 || d->n_kv_heads < 1 || d->n_q_heads % d->n_kv_heads != 0)
-        return QSA_ERR_INVALID_ARG;
-    if (d->block_size != kBlock || d->top_k != kTopK || d->kv_capacity <= 0 || d->kv_capacity % kBlock != 0 ||
-        d->kv_capacity >= (1ll << 31) || !std::isfinite(d->softmax_scale) || n_q < 0)
-        return QSA_ERR_INVALID_ARG;
-    if (d->head_dim != kHeadDim || d->n_idx_heads != kIdxHeads || d->idx_dim != kIdxDim ||
-        d->n_q_heads / d->n_kv_heads > kMaxGroup || n_q > 65535)
-        return QSA_ERR_UNSUPPORTED;
-    return QSA_OK;
 }
 
 }  // namespace
@@ -81,9 +75,10 @@ extern "C" int qsa_sparse_attn_noalloc(const qsa_dims* dims, const void* q, cons
                                        const int32_t* sel_idx, const int32_t* sel_cnt, int32_t n_q, void* out,
                                        void* stream)
 {
-    // same argument rules as qsa_sparse_attn, minus the workspace
-    const int rc = check_args(dims, n_q);
+    // same argument rules as qsa_sparse_attn (the shared checks), minus the workspace
+    int rc = check_dims(dims);
     if (rc != QSA_OK) return rc;
+    if ((rc = check_rows(dims, n_q, 0)) != QSA_OK) return rc;
     if (n_q == 0) return QSA_OK;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(q_seq) || !aligned16(q_pos) ||
         !aligned16(sel_idx) || !aligned16(sel_cnt) || !aligned16(out))
@@ -96,9 +91,9 @@ extern "C" int qsa_sparse_attn_noalloc(const qsa_dims* dims, const void* q, cons
         n_split > 1 ? (size_t)n_q * dims->n_kv_heads * n_split * (32 + 16 * kHeadDim) * 4 : 0;
     if (counter_bytes + partial_bytes > kScratchBytes) return QSA_ERR_WORKSPACE_TOO_SMALL;
 
-    void* base = nullptr;
-    if (scratch_address(&base) != cudaSuccess) return QSA_ERR_CUDA;
     cudaStream_t st = (cudaStream_t)stream;
+    void* base = nullptr;
+    if (scratch_address(st, &base) != cudaSuccess) return QSA_ERR_CUDA;
     unsigned* counters = (unsigned*)base;
     float* partial = (float*)((char*)base + counter_bytes);
     if (n_split > 1 && cudaMemsetAsync(counters, 0, (size_t)n_q * dims->n_kv_heads * 4, st) != cudaSuccess)

@@ -118,6 +118,14 @@ struct WsLayout {
     int n_split = 1;
 };
 
+// ---- host-side argument checks shared by every entry point (api.cu) ----
+// Pointer non-null and 16-byte aligned.
+bool aligned16(const void* p);
+// The dims every call needs: sizes, fixed method parameters, supported head layout.
+int check_dims(const qsa_dims* d);
+// Query count and candidate-block bound of a call.
+int check_rows(const qsa_dims* d, int32_t n_q, int64_t max_blocks);
+
 // Chunk of candidate blocks one CTA of the decode scoring/select passes handles.
 int select_chunk(int64_t max_blocks, int32_t n_rows);
 // Split-K factor of the decode attention.

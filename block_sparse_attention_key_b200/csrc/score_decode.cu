@@ -13,9 +13,10 @@
 // therefore run on mma.sync (m16n8k16, bf16 in, fp32 accumulate): 16 blocks x 16
 // dims of pooled keys as A, the query's 4 indexer heads (plus 4 zero columns) as
 // B, four K-steps per 16 blocks.  Pooled tiles of 128 blocks (16 KiB) stream
-// through a 4-deep cp.async ring into XOR-swizzled shared memory (64 KiB in flight
-// per CTA, one wave of CTAs); each of the 8 warps takes 16 blocks of a tile.  The
-// epilogue applies ReLU and the head weights with one fp32 FMA chain per block
+// through a 4-slot cp.async ring into XOR-swizzled shared memory (three tiles in
+// flight per CTA while the fourth is read, one wave of CTAs); each of the 8 warps
+// takes 16 blocks of a tile.  A slot is refilled only after the barrier that
+// follows every warp's reads of it.  The epilogue applies ReLU and the head weights with one fp32 FMA chain per block
 // (w0*r0, then + w1*r1, + w2*r2, + w3*r3).  fp32 accumulation of bf16 x bf16
 // products is exact for small integers.  Optionally the same pass histograms the
 // scores' top key digit for the select.
@@ -29,7 +30,7 @@ namespace qsa {
 namespace {
 
 constexpr int kTile = 128;                       // pooled blocks per stage
-constexpr int kStages = 4;                       // stages in flight per CTA
+constexpr int kStages = 4;                       // ring slots per CTA
 constexpr int kTileBytes = kTile * kIdxDim * 2;  // 16 KiB
 constexpr int kRingBytes = kStages * kTileBytes;  // 64 KiB
 // dynamic shared memory: the copy ring, later (in a row's last CTA) the row's keys
@@ -143,10 +144,13 @@ k_score_decode(const uint4* __restrict__ q_idx, const float* __restrict__ w, con
         const int m = lane >> 3;
 
         for (int tl = 0; tl < n_tiles; ++tl) {
+            // tiles tl .. tl + kStages - 2 are committed: wait for tile tl, then the
+            // barrier both publishes every thread's copies of tile tl and ensures every
+            // warp has finished reading tile tl - 1, whose slot the next issue reuses
+            cp_async_wait<kStages - 2>();
+            __syncthreads();
             if (tl + kStages - 1 < n_tiles) issue(tl + kStages - 1);
             cp_async_commit();
-            cp_async_wait<kStages - 1>();
-            __syncthreads();  // every thread's copies of tile tl have landed
             const uint32_t tbase = sbase + (uint32_t)((tl % kStages) * kTileBytes);
             float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll

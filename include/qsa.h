@@ -164,8 +164,9 @@ int qsa_sparse_attn(const qsa_dims* dims, const void* q, const void* k_cache, co
  * 2.5 MiB of partials; one needing more than 16 MiB (more than about 4 million
  * pairs) returns QSA_ERR_WORKSPACE_TOO_SMALL before launching.
  * The first call on each device, with that device current, looks the array's
- * device address up (cudaGetSymbolAddress); make that first call before any
- * stream capture.  All calls share the array: counters are cleared at the start
+ * device address up (cudaGetSymbolAddress), and so does every later call made
+ * outside stream capture (a device reset may move the array); make that first
+ * call before any stream capture.  All calls share the array: counters are cleared at the start
  * of each call, and calls whose executions overlap on the GPU race on it.  No
  * device status word: out-of-range indices are skipped but not reported.
  * Nothing in this call allocates memory. */

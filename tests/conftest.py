@@ -10,6 +10,16 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+    config._qsa_notes = []
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Print what the parity tests measured about themselves (rows checked, wall time, cores)."""
+    notes = getattr(config, "_qsa_notes", [])
+    if notes:
+        terminalreporter.section("QSA parity notes")
+        for n in notes:
+            terminalreporter.write_line(n)
 
 
 @pytest.fixture(scope="session")

@@ -1,7 +1,9 @@
 """Parity of the whole layer on the five synthetic workloads, in the launch
 configuration the benchmark times: every row's selection checked for its
-invariants, and the oracle's selection and output compared on every row
-(decode) or on a stratified sample of rows (prefill chunks)."""
+invariants and compared bit for bit with the oracle's on every row (prefill
+chunks: the oracle's per-row scoring and top-512 spread over the host's cores),
+and the attention output compared with the oracle's on every row (decode) or on
+a stratified sample of rows (prefill chunks)."""
 
 import numpy as np
 import pytest
@@ -11,6 +13,7 @@ from oracle import oracle as O
 from qsa_synth import workloads as W
 
 import gpu_util as gu
+import oracle_parallel as OP
 
 pytestmark = pytest.mark.gpu
 
@@ -32,7 +35,7 @@ def sample_rows(n, k=24, seed=0):
 
 
 @pytest.mark.parametrize("cid", [0, 1, 2, 3, 4])
-def test_workload_parity(cid):
+def test_workload_parity(cid, request):
     from qsa_synth import device as sdev
     wl = W.by_id(cid)
     dw = sdev.DeviceWorkload(wl)
@@ -46,6 +49,15 @@ def test_workload_parity(cid):
         rows = list(range(n)) if wl.mode == "decode" else sample_rows(n, seed=cid)
         sel = sel_idx.cpu().numpy()
         cnt = sel_cnt.cpu().numpy()
+        if wl.mode == "prefill":
+            # selection of every row of the chunk against the oracle, rows shared out over the cores
+            want_all, secs, procs = OP.oracle_selections(wl, step)
+            assert len(want_all) == n
+            for r in range(n):
+                np.testing.assert_array_equal(sel[r, : cnt[r]], want_all[r], err_msg=f"{wl.name} step {step} row {r}")
+            request.config._qsa_notes.append(
+                f"{wl.name}: selection of all {n} rows bit-exact vs the oracle "
+                f"({secs:.1f} s wall on {procs} host cores)")
         got = gu.bf16_to_f64(out[rows])
         want = np.zeros_like(got)
         for j, r in enumerate(rows):

@@ -412,12 +412,19 @@ def test_forward_decode_ties_take_lowest_blocks(cap):
         z = torch.zeros_like(t)
         z[:, :, 0] = t[:, :, 0]
         return z
-    sel, cnt, flags, (dw, T) = _prefill_run(wl, q_idx_override=one_dim, mode=0, return_inputs=True)
+    sel, cnt, flags = _prefill_run(wl, q_idx_override=one_dim, mode=0)
     assert flags == 0
-    q_bits = gu.to_bits(one_dim(T["q_idx"]))
-    w = T["w"].cpu().numpy()
+    # expected values from the host generator and the oracle alone (nothing read back
+    # from the device): pooled keys by the oracle's pooling, indexer queries with every
+    # dimension but the first of each head zeroed
+    import qsa_synth as syn
+    wo = O.WorkloadOracle(wl)
+    st = wl.steps[0]
+    q_bits = syn.gen_q_idx(wl.seed, st.query_ids, wl.n_idx_heads, wl.idx_dim).copy()
+    q_bits[:, :, 1:] = 0
+    w = syn.gen_w(wl.seed, st.query_ids, wl.n_idx_heads)
     for r in range(3):
-        pooled_bits = gu.to_bits(dw.pooled[r, :n_c])
+        pooled_bits = wo.pooled(st.q_seq[r], n_c)
         want = O.select_top_blocks(O.block_scores(q_bits[r], w[r], pooled_bits))
         assert cnt[r] == len(want)
         np.testing.assert_array_equal(sel[r, : cnt[r]], want, err_msg=f"row {r}")
