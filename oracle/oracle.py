@@ -55,6 +55,9 @@ def lib():
         L.qo_select_top_blocks.restype = ctypes.c_int32
         L.qo_attended_tokens.argtypes = [_i32p, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, _i64p]
         L.qo_attended_tokens.restype = ctypes.c_int64
+        L.qo_attended_tokens_shared.argtypes = [_i32p, ctypes.c_int32, ctypes.c_int64, ctypes.c_int64,
+                                                ctypes.c_int32, _i64p]
+        L.qo_attended_tokens_shared.restype = ctypes.c_int64
         L.qo_gqa_attention.argtypes = [_u16p, _u16p, _u16p, ctypes.c_int64, ctypes.c_int32,
                                        ctypes.c_int32, ctypes.c_int32, ctypes.c_double, _f64p]
         L.qo_gqa_attention.restype = None
@@ -113,6 +116,18 @@ def attended_tokens(sel, t, block_size=4):
     buf = np.zeros(sel.size * block_size + block_size, dtype=np.int64)
     n = lib().qo_attended_tokens(sel if sel.size else np.zeros(1, np.int32), sel.size, int(t),
                                  block_size, buf)
+    return buf[:n].copy()
+
+
+def attended_tokens_shared(sel, t_sel, t, block_size=4):
+    """Step 4 for a draft query at ``t`` reusing the selection made at ``t_sel``:
+    the selected blocks' tokens, then every token from the selection query's first
+    incomplete block up to ``t``."""
+    sel = np.ascontiguousarray(sel, dtype=np.int32)
+    tail = int(t) + 1 - ((int(t_sel) + 1) // block_size) * block_size
+    buf = np.zeros(sel.size * block_size + max(tail, 0) + 1, dtype=np.int64)
+    n = lib().qo_attended_tokens_shared(sel if sel.size else np.zeros(1, np.int32), sel.size, int(t_sel), int(t),
+                                        block_size, buf)
     return buf[:n].copy()
 
 

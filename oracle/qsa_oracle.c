@@ -125,6 +125,19 @@ int64_t qo_attended_tokens(const int32_t* sel, int32_t cnt, int64_t t, int32_t b
     return n;
 }
 
+int64_t qo_attended_tokens_shared(const int32_t* sel, int32_t cnt, int64_t t_sel, int64_t t,
+                                  int32_t block_size, int64_t* tokens)
+{
+    int64_t n = 0;
+    for (int32_t i = 0; i < cnt; ++i)
+        for (int32_t j = 0; j < block_size; ++j)
+            tokens[n++] = (int64_t)sel[i] * block_size + j;
+    /* everything after the complete blocks the selection was made over, up to t */
+    const int64_t n_complete_sel = (t_sel + 1) / block_size;
+    for (int64_t p = n_complete_sel * block_size; p <= t; ++p) tokens[n++] = p;
+    return n;
+}
+
 void qo_gqa_attention(const uint16_t* q, const uint16_t* k_rows, const uint16_t* v_rows,
                       int64_t n_tok, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
                       double scale, double* out)

@@ -62,6 +62,16 @@ int32_t qo_select_top_blocks(const double* scores, int64_t n_cand, int32_t top_k
 int64_t qo_attended_tokens(const int32_t* sel, int32_t cnt, int64_t t, int32_t block_size,
                            int64_t* tokens);
 
+/* Step 4, multi-token decode.  keieiax.jp glossary "Qwen Sparse Attention", FAQ on
+ * multi-token prediction: the selected top blocks are reused between the
+ * speculative steps.  A draft query at position t that reuses the selection made
+ * for the query at t_sel (t_sel <= t) attends the tokens of the selected blocks,
+ * then every token from the selection query's first incomplete block,
+ * block_size*floor((t_sel+1)/block_size), up to t.  With t == t_sel this is
+ * qo_attended_tokens.  Writes ascending token positions and returns how many. */
+int64_t qo_attended_tokens_shared(const int32_t* sel, int32_t cnt, int64_t t_sel, int64_t t,
+                                  int32_t block_size, int64_t* tokens);
+
 /* Step 5.  For each query head h (KV head h / (n_q_heads/n_kv_heads)):
  * out[h][:] = sum_j softmax_j(scale * q[h].k[j]) v[j].
  * q is [n_q_heads][head_dim]; k_rows and v_rows are [n_tok][n_kv_heads][head_dim]. */

@@ -3,7 +3,8 @@
 Each case plants one mistake in a copy of the C oracle (a wrong head map, a dropped
 ReLU, an off-by-one block count, the wrong tie order, a wrong mean divisor, a
 transposed indexer query, a missing softmax scale, a dropped partial-block token,
-ties rounded away from even) and runs the CPU pins against the copy: every planted
+ties rounded away from even, a draft query's tail starting at its own block or
+ending at the selection's query) and runs the CPU pins against the copy: every planted
 mistake must make them fail.  Only the copy under a temporary directory is changed.
 """
 
@@ -28,6 +29,10 @@ MUTATIONS = [
     ("partial block token", "for (int64_t p = n_complete * block_size; p <= t; ++p)",
      "for (int64_t p = n_complete * block_size; p < t; ++p)"),
     ("ties to even", "const double r = nearbyint(a / step);", "const double r = floor(a / step + 0.5);"),
+    ("draft tail start", "const int64_t n_complete_sel = (t_sel + 1) / block_size;",
+     "const int64_t n_complete_sel = (t + 1) / block_size;"),
+    ("draft tail end", "for (int64_t p = n_complete_sel * block_size; p <= t; ++p)",
+     "for (int64_t p = n_complete_sel * block_size; p <= t_sel; ++p)"),
 ]
 
 

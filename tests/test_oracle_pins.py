@@ -304,3 +304,60 @@ def test_workload_query_selection_by_brute_force(oracle_lib):
     order = np.lexsort((np.arange(2048), -scores))[:512]
     assert sel.tolist() == sorted(order.tolist())
     assert out.shape == (8, 128) and np.isfinite(out).all()
+
+
+# ------------------------------------------------------------------ multi-token decode (shared selection)
+
+def test_shared_tokens_closed_forms(oracle_lib):
+    """A draft query reusing the selection made at t_sel attends the selected blocks
+    plus every token from the selection's first incomplete block up to itself."""
+    o = oracle_lib
+    # same position: the ordinary rule
+    for sel, t in ([[0, 2], 11], [[1], 9], [[], 2], [[0], 3]):
+        s = np.array(sel, np.int32)
+        assert o.attended_tokens_shared(s, t, t).tolist() == o.attended_tokens(s, t).tolist()
+    # selection at t_sel = 9 (2 complete blocks, partial block {8, 9}); drafts at 10, 11, 12, 13
+    s = np.array([0], np.int32)
+    assert o.attended_tokens_shared(s, 9, 10).tolist() == [0, 1, 2, 3, 8, 9, 10]
+    assert o.attended_tokens_shared(s, 9, 11).tolist() == [0, 1, 2, 3, 8, 9, 10, 11]
+    # draft 12 completes nothing new for the selection: block 2 (8..11) was not a candidate at t_sel
+    assert o.attended_tokens_shared(s, 9, 12).tolist() == [0, 1, 2, 3, 8, 9, 10, 11, 12]
+    assert o.attended_tokens_shared(s, 9, 13).tolist() == [0, 1, 2, 3, 8, 9, 10, 11, 12, 13]
+    # t_sel = 11 completes block 2: the tail starts at 12
+    s = np.array([2], np.int32)
+    assert o.attended_tokens_shared(s, 11, 13).tolist() == [8, 9, 10, 11, 12, 13]
+
+
+@pytest.mark.parametrize("t_sel,draft", [(40, 1), (41, 2), (43, 3), (102, 4)])
+def test_shared_tokens_invariants(oracle_lib, t_sel, draft):
+    """Counts, causality and coverage, for random selections below t_sel."""
+    o = oracle_lib
+    rng = np.random.default_rng(t_sel * 10 + draft)
+    n_c = (t_sel + 1) // 4
+    sel = np.sort(rng.choice(n_c, size=min(5, n_c), replace=False)).astype(np.int32)
+    t = t_sel + draft
+    toks = o.attended_tokens_shared(sel, t_sel, t)
+    assert (np.diff(toks) > 0).all() and toks.max() == t and (toks <= t).all()
+    assert len(toks) == 4 * len(sel) + (t + 1 - 4 * n_c)
+    covered = set(toks.tolist())
+    for b in range(n_c):  # a complete block below t_sel is attended whole or not at all
+        inside = [p in covered for p in range(4 * b, 4 * b + 4)]
+        assert all(inside) == (b in sel.tolist()) and (any(inside) == all(inside))
+    assert all(p in covered for p in range(4 * n_c, t + 1))
+
+
+@pytest.mark.parametrize("t_sel,draft", [(8, 1), (10, 3), (2047, 2), (2045, 4)])
+def test_shared_selection_below_budget_is_dense_causal_gqa(oracle_lib, t_sel, draft):
+    """With <= 512 complete blocks at t_sel every block is selected, so each draft
+    query at t_sel + j attends tokens 0..t_sel+j: dense causal GQA (fp64 SDPA)."""
+    o = oracle_lib
+    t_last = t_sel + draft
+    inp = _dense_inputs(70 + t_sel + draft, t_last + 1, 8, 2, 32)
+    pooled = o.pool_blocks(inp["idx_k"])
+    n_c = (t_sel + 1) // 4
+    sel = o.select_top_blocks(o.block_scores(inp["q_idx"], inp["w"], pooled[:n_c]))
+    assert sel.tolist() == list(range(n_c))
+    for t in range(t_sel, t_last + 1):
+        toks = o.attended_tokens_shared(sel, t_sel, t)
+        out = o.gqa_attention(inp["q"], inp["k"][toks], inp["v"][toks])
+        np.testing.assert_allclose(out, _sdpa(inp["q"], inp["k"][: t + 1], inp["v"][: t + 1]), rtol=0, atol=1e-12)
