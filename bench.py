@@ -36,8 +36,11 @@ def parse():
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    p.add_argument("--workload", default="decode_64k_b16")
+    p.add_argument("--workload", default="decode_64k_b16",
+                   help="headline configuration (the others are measured after it unless --no-workload-map)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-workload-map", dest="workload_map", action="store_false",
+                   help="skip the other configurations' measurements")
     return p.parse_args()
 
 
@@ -236,229 +239,367 @@ def job_tokens_per_s(world, tokens_per_rank, ms_per_step):
     return world * tokens_per_rank / (ms_per_step / 1e3)
 
 
-def run_ours(args, wl):
-    import torch
-    import torch.distributed as dist
-    import block_sparse_attention_key_b200 as qsa
-    from block_sparse_attention_key_b200 import build as qbuild
-    from qsa_synth import device as sdev
+def attended_tokens_of(wl, step, cnt):
+    """Tokens each query attends: 4 per selected block plus its partial block."""
+    part = (np.asarray(wl.steps[step].q_pos, dtype=np.int64) + 1) % wl.block_size
+    return np.asarray(cnt, dtype=np.int64) * wl.block_size + part
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+def attn_bytes_of(wl, toks):
+    """Algorithmic bytes of gathered attention: K+V rows of every attended token for
+    every KV head, q read and out written."""
+    n_q = len(toks)
+    return int(toks.sum() * wl.n_kv_heads * wl.head_dim * 2 * 2 + 2 * n_q * wl.n_q_heads * wl.head_dim * 2)
 
-    def max_ms(x):
-        return max_over_ranks(x, world, "cuda")
 
-    if rank == 0:
-        qbuild.build()
-        sdev.build()
-    barrier()
-    qsa.load()
+def select_work_of(wl, step):
+    """(flops, bytes) of indexer scoring for one step: 4 heads x 64 dims x 2 flops per
+    (query, complete causal block), 128 B of pooled key per (query, block) read."""
+    n_c = (np.asarray(wl.steps[step].q_pos, dtype=np.int64) + 1) // wl.block_size
+    return int(n_c.sum() * wl.n_idx_heads * wl.idx_dim * 2), int(n_c.sum() * wl.idx_dim * 2)
 
-    mode = qsa.QSA_MODE_PREFILL if wl.mode == "prefill" else qsa.QSA_MODE_DECODE
-    dims = qsa.make_dims(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.kv_capacity)
-    dw = sdev.DeviceWorkload(wl)
-    # history: every block completed before the first step is already pooled
-    st0 = wl.steps[0]
-    zeros = torch.zeros(wl.batch, dtype=torch.int32, device="cuda")
-    qsa.qsa_pool_block_keys(dims, dw.idx_k, dw.pooled, zeros,
-                            torch.tensor(st0.len_before, dtype=torch.int32, device="cuda"), max(st0.len_before))
-    steps = [dw.step_tensors(i) for i in range(len(wl.steps))]
-    n_q_unit = sum(T["n_q"] for T in steps)
-    ws_bytes = max(qsa.qsa_workspace_bytes(dims, T["n_q"], T["max_blocks"], mode) for T in steps)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
-    qsa.qsa_workspace_init(ws)
-    outs = [torch.empty((T["n_q"], wl.n_q_heads, wl.head_dim), dtype=torch.bfloat16, device="cuda") for T in steps]
-    sels = [torch.empty((T["n_q"], wl.top_k), dtype=torch.int32, device="cuda") for T in steps]
-    cnts = [torch.empty((T["n_q"],), dtype=torch.int32, device="cuda") for T in steps]
-    # L2 flush: write one buffer larger than L2, then read another, so L2 ends up
-    # full of clean lines that belong to neither the inputs nor the outputs
-    flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
-    flush_sink = torch.empty((), dtype=torch.float32, device="cuda")
 
-    def flush():
-        flush_w.fill_(1)
-        torch.sum(flush_r, dim=0, out=flush_sink)
+class Env:
+    """Per-rank GPU state shared by the workload measurements."""
 
-    def forward(T, out, sel, cnt, src=None):
-        src = src or T
-        qsa.qsa_forward(dims, q=src["q"], k_cache=dw.k_cache, v_cache=dw.v_cache, idx_k=dw.idx_k, pooled=dw.pooled,
-                        q_idx=src["q_idx"], w=src["w"], len_before=src["len_before"], len_after=src["len_after"],
-                        q_seq=src["q_seq"], q_pos=src["q_pos"], n_q=T["n_q"], max_new_tokens=T["max_new_tokens"],
-                        max_blocks=T["max_blocks"], mode=mode, out=out, workspace=ws, sel_idx=sel, sel_cnt=cnt)
+    def __init__(self, args):
+        import torch
+        import torch.distributed as dist
+        import block_sparse_attention_key_b200 as qsa
+        from block_sparse_attention_key_b200 import build as qbuild
+        from qsa_synth import device as sdev
+        self.torch, self.dist, self.qsa, self.sdev = torch, dist, qsa, sdev
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        if self.world != args.gpus:
+            raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={self.world}")
+        torch.cuda.set_device(self.local)
+        if self.world > 1:
+            import datetime
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+        if self.rank == 0:
+            qbuild.build()
+            sdev.build()
+        self.barrier()
+        qsa.load()
+        # L2 flush: write one buffer larger than L2, then read another, so L2 ends up
+        # full of clean lines that belong to neither the inputs nor the outputs
+        self.flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        self.flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+        self.flush_sink = torch.empty((), dtype=torch.float32, device="cuda")
 
-    def unit():
-        """One unit of work: every step of the workload (one step for most workloads)."""
-        for T, out, sel, cnt in zip(steps, outs, sels, cnts):
-            forward(T, out, sel, cnt)
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
 
-    def timed(fn, k):
+    def max_ms(self, x):
+        return max_over_ranks(x, self.world, "cuda")
+
+    def flush(self):
+        self.flush_w.fill_(1)
+        self.torch.sum(self.flush_r, dim=0, out=self.flush_sink)
+
+    def timed(self, fn, k):
+        """k timed calls of fn, each after an L2 flush, CUDA events on the current stream."""
+        torch = self.torch
         stream = torch.cuda.current_stream()
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
         for a, b in evs:
-            flush()
+            self.flush()
             a.record(stream)
             fn()
             b.record(stream)
         torch.cuda.synchronize()
         return [a.elapsed_time(b) for a, b in evs]
 
-    for _ in range(max(args.warmup, 3)):
-        unit()
-    torch.cuda.synchronize()
-    flags = qsa.qsa_read_device_status(ws)
-    if flags:
-        raise SystemExit(f"device status flags {flags:#x} after warm-up")
-    # the step as a CUDA graph: all lengths and positions are device-side, so it replays as is
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        unit()
-    for _ in range(3):
-        graph.replay()
-    torch.cuda.synchronize()
 
-    clocks = Clocks(local) if rank == 0 else None
+class Bench:
+    """One workload resident in HBM: its caches, step inputs, workspace and outputs."""
+
+    def __init__(self, env, wl):
+        torch, qsa, sdev = env.torch, env.qsa, env.sdev
+        self.env, self.wl = env, wl
+        self.mode = qsa.QSA_MODE_PREFILL if wl.mode == "prefill" else qsa.QSA_MODE_DECODE
+        self.dims = qsa.make_dims(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.kv_capacity)
+        self.dw = sdev.DeviceWorkload(wl)
+        st0 = wl.steps[0]
+        zeros = torch.zeros(wl.batch, dtype=torch.int32, device="cuda")
+        # history: every block completed before the first step is already pooled
+        qsa.qsa_pool_block_keys(self.dims, self.dw.idx_k, self.dw.pooled, zeros,
+                                torch.tensor(st0.len_before, dtype=torch.int32, device="cuda"), max(st0.len_before))
+        self.steps = [self.dw.step_tensors(i) for i in range(len(wl.steps))]
+        self.n_q_unit = sum(T["n_q"] for T in self.steps)
+        ws_bytes = max(qsa.qsa_workspace_bytes(self.dims, T["n_q"], T["max_blocks"], self.mode) for T in self.steps)
+        self.ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+        qsa.qsa_workspace_init(self.ws)
+        self.outs = [torch.empty((T["n_q"], wl.n_q_heads, wl.head_dim), dtype=torch.bfloat16, device="cuda")
+                     for T in self.steps]
+        self.sels = [torch.empty((T["n_q"], qsa.QSA_SEL_CAP), dtype=torch.int32, device="cuda") for T in self.steps]
+        self.cnts = [torch.empty((T["n_q"],), dtype=torch.int32, device="cuda") for T in self.steps]
+
+    def forward(self, T, out, sel, cnt, src=None):
+        src = src or T
+        dw = self.dw
+        self.env.qsa.qsa_forward(
+            self.dims, q=src["q"], k_cache=dw.k_cache, v_cache=dw.v_cache, idx_k=dw.idx_k, pooled=dw.pooled,
+            q_idx=src["q_idx"], w=src["w"], len_before=src["len_before"], len_after=src["len_after"],
+            q_seq=src["q_seq"], q_pos=src["q_pos"], n_q=T["n_q"], max_new_tokens=T["max_new_tokens"],
+            max_blocks=T["max_blocks"], mode=self.mode, out=out, workspace=self.ws, sel_idx=sel, sel_cnt=cnt)
+
+    def unit(self):
+        """One unit of work: every step of the workload (one step for most workloads)."""
+        for T, out, sel, cnt in zip(self.steps, self.outs, self.sels, self.cnts):
+            self.forward(T, out, sel, cnt)
+
+    def step_timing(self, args):
+        """The unit as a CUDA graph (all lengths and positions are device-side), K timed
+        replays with L2 flushed before each; returns (ms per unit, eager ms, graph)."""
+        env, torch, qsa = self.env, self.env.torch, self.env.qsa
+        for _ in range(max(args.warmup, 3)):
+            self.unit()
+        torch.cuda.synchronize()
+        flags = qsa.qsa_read_device_status(self.ws)
+        if flags:
+            raise SystemExit(f"{self.wl.name}: device status flags {flags:#x} after warm-up")
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.unit()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        ms = env.max_ms(float(np.mean(env.timed(graph.replay, args.steps))))
+        ms_eager = env.max_ms(float(np.mean(env.timed(self.unit, args.steps))))
+        return ms, ms_eager, graph
+
+    def kernels(self, args, hbm_peak, tc_peak, peak_kind, attn_sets):
+        """Standalone timing of the two hot steps of the last step's inputs:
+        selection (qsa_select_blocks: scores + top-512) and gathered attention
+        (qsa_sparse_attn, the kernel the forward runs for this shape).  Decode
+        attention is timed as `attn_sets` back-to-back launches on distinct query
+        sets (distinct selections, so no launch finds another's rows in L2) in one
+        CUDA graph, L2 flushed before each replay; per-launch time = replay / sets."""
+        env, torch, qsa, sdev, wl = self.env, self.env.torch, self.env.qsa, self.env.sdev, self.wl
+        si = len(self.steps) - 1
+        T = self.steps[si]
+        n_q, mb = T["n_q"], T["max_blocks"]
+        res = {}
+        sel = torch.empty((n_q, qsa.QSA_SEL_CAP), dtype=torch.int32, device="cuda")
+        cnt = torch.empty((n_q,), dtype=torch.int32, device="cuda")
+        run_sel = lambda: qsa.qsa_select_blocks(self.dims, T["q_idx"], T["w"], self.dw.pooled, T["q_seq"],
+                                                 T["q_pos"], n_q, mb, self.mode, sel, cnt, self.ws)
+        run_sel()
+        sel_ms = env.max_ms(float(np.mean(env.timed(run_sel, args.steps))))
+        assert torch.equal(sel, self.sels[si]) and torch.equal(cnt, self.cnts[si])
+        flops, pbytes = select_work_of(wl, si)
+        res["select_us"] = 1e3 * sel_ms
+        if self.mode == qsa.QSA_MODE_PREFILL:
+            ach = flops / (sel_ms / 1e3) / 1e12
+            res["roofline_select"] = {"kernels": "k_prefill_scores_tc (sampling + main), k_prefill_finish, "
+                                                 "k_prefill_fallback", "bound": "tensor",
+                                      "achieved": round(ach, 1), "peak": tc_peak, "unit": "TFLOP/s",
+                                      "frac": round(ach / tc_peak, 4),
+                                      "peak_source": f"{peak_kind} bf16_tflops (burst)", "flops_per_call": flops}
+        else:
+            ach = pbytes / (sel_ms / 1e3) / 1e9
+            res["roofline_select"] = {"kernels": "k_score_decode (+ k_topk_collect beyond 16,384 blocks)",
+                                      "bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s",
+                                      "frac": round(ach / hbm_peak, 4),
+                                      "peak_source": f"{peak_kind} hbm_gbs (burst copy)",
+                                      "algorithmic_bytes_per_call": pbytes}
+
+        # attention: `sets` query sets with their own selections
+        sets = attn_sets if self.mode == qsa.QSA_MODE_DECODE else 1
+        qs, sels, cnts, nbytes = [T["q"]], [self.sels[si]], [self.cnts[si]], 0
+        toks = attended_tokens_of(wl, si, self.cnts[si].cpu().numpy())
+        nbytes += attn_bytes_of(wl, toks)
+        for r in range(1, sets):
+            q = torch.empty_like(T["q"])
+            q_idx = torch.empty_like(T["q_idx"])
+            w = torch.empty_like(T["w"])
+            qid0 = 1_000_000 * r
+            sdev.fill_q(q, wl.seed, qid0)
+            sdev.fill_q_idx(q_idx, wl.seed, qid0)
+            sdev.fill_w(w, wl.seed, qid0)
+            s_r = torch.empty_like(sel)
+            c_r = torch.empty_like(cnt)
+            qsa.qsa_select_blocks(self.dims, q_idx, w, self.dw.pooled, T["q_seq"], T["q_pos"], n_q, mb, self.mode,
+                                  s_r, c_r, self.ws)
+            qs.append(q)
+            sels.append(s_r)
+            cnts.append(c_r)
+            nbytes += attn_bytes_of(wl, attended_tokens_of(wl, si, c_r.cpu().numpy()))
+        out_k = torch.empty_like(self.outs[si])
+
+        def attn_all():
+            for q, s_r, c_r in zip(qs, sels, cnts):
+                qsa.qsa_sparse_attn(self.dims, q, self.dw.k_cache, self.dw.v_cache, T["q_seq"], T["q_pos"], s_r,
+                                    c_r, n_q, out_k, self.ws)
+        attn_all()
+        torch.cuda.synchronize()
+        # the first set is the forward's own query set: same output
+        qsa.qsa_sparse_attn(self.dims, qs[0], self.dw.k_cache, self.dw.v_cache, T["q_seq"], T["q_pos"], sels[0],
+                            cnts[0], n_q, out_k, self.ws)
+        res["attn_matches_forward"] = bool(torch.equal(out_k, self.outs[si]))
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            attn_all()
+        g.replay()
+        torch.cuda.synchronize()
+        attn_ms = env.max_ms(float(np.mean(env.timed(g.replay, args.steps)))) / sets
+        del g
+        res["attn_us"] = 1e3 * attn_ms
+        res["attn_sets_per_graph"] = sets
+        ach = (nbytes / sets) / (attn_ms / 1e3) / 1e9
+        res["roofline_attention"] = {
+            "kernel": "k_attn_decode" if self.mode == qsa.QSA_MODE_DECODE else "k_sparse_attn", "bound": "hbm",
+            "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s", "frac": round(ach / hbm_peak, 4),
+            "peak_source": f"{peak_kind} hbm_gbs (burst copy)", "algorithmic_bytes_per_launch": int(nbytes / sets)}
+        if self.mode == qsa.QSA_MODE_PREFILL:
+            # a block chosen by several queries of the chunk is gathered once per query
+            blocks = torch.cat([s_r[s_r >= 0] for s_r in sels]).unique().numel()
+            res["roofline_attention"]["unique_bytes"] = int(blocks * wl.block_size * wl.n_kv_heads * wl.head_dim * 4)
+        return res
+
+    def e2e(self, args):
+        """End to end: host buffers in, host buffer out, copies inside the timed region.
+        Every step's inputs travel in one pinned host buffer: queries, indexer inputs,
+        positions, and the appended tokens' K/V rows and indexer keys, which are
+        scattered into the caches on the device."""
+        env, torch, dw = self.env, self.env.torch, self.dw
+        e2e_steps = []
+        for si, T in enumerate(self.steps):
+            st = self.wl.steps[si]
+            parts = {k: T[k] for k in ("q", "q_idx", "w", "len_before", "len_after", "q_seq", "q_pos")}
+            new = [(s, a, b) for s, (a, b) in enumerate(zip(st.len_before, st.len_after)) if b > a]
+            seq_i = torch.tensor([s for s, a, b in new for _ in range(a, b)], dtype=torch.int64, device="cuda")
+            pos_i = torch.tensor([p for s, a, b in new for p in range(a, b)], dtype=torch.int64, device="cuda")
+            parts["k_new"] = dw.k_cache[seq_i, :, pos_i].contiguous()
+            parts["v_new"] = dw.v_cache[seq_i, :, pos_i].contiguous()
+            parts["ik_new"] = dw.idx_k[seq_i, pos_i].contiguous()
+            layout, off = {}, 0
+            for k, v in parts.items():
+                nb = v.numel() * v.element_size()
+                layout[k] = (off, nb, v.dtype, tuple(v.shape))
+                off += (nb + 255) // 256 * 256
+            h_in = torch.empty(off, dtype=torch.uint8).pin_memory()
+            for k, v in parts.items():
+                o, nb, _, _ = layout[k]
+                h_in[o:o + nb].copy_(v.reshape(-1).view(torch.uint8).cpu())
+            d_in = torch.empty(off, dtype=torch.uint8, device="cuda")
+            view = {k: d_in[o:o + nb].view(dt).view(shape) for k, (o, nb, dt, shape) in layout.items()}
+            h_out = torch.empty(tuple(self.outs[si].shape), dtype=self.outs[si].dtype).pin_memory()
+            e2e_steps.append((T, h_in, d_in, view, seq_i, pos_i, h_out))
+
+        def unit_e2e():
+            for (T, h_in, d_in, view, seq_i, pos_i, h_out), out, sel, cnt in zip(e2e_steps, self.outs, self.sels,
+                                                                                  self.cnts):
+                d_in.copy_(h_in, non_blocking=True)
+                dw.k_cache[seq_i, :, pos_i] = view["k_new"]
+                dw.v_cache[seq_i, :, pos_i] = view["v_new"]
+                dw.idx_k[seq_i, pos_i] = view["ik_new"]
+                self.forward(T, out, sel, cnt, src=view)
+                h_out.copy_(out, non_blocking=True)
+
+        for _ in range(3):
+            unit_e2e()
+        torch.cuda.synchronize()
+        graph_e2e = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_e2e):
+            unit_e2e()
+        e2e_ms = []
+        for _ in range(args.steps):
+            env.flush()
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            graph_e2e.replay()
+            torch.cuda.current_stream().synchronize()
+            e2e_ms.append(1e3 * (time.perf_counter() - t0))
+        del graph_e2e
+        e2e_ms = env.max_ms(float(np.mean(e2e_ms)))
+        h2d = sum(x[1].numel() for x in e2e_steps)
+        d2h = sum(x[6].numel() * x[6].element_size() for x in e2e_steps)
+        return {"value": job_tokens_per_s(env.world, self.n_q_unit, e2e_ms), "unit": "tokens/s",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "timing": "host wall clock around one CUDA-graph replay of: one H2D copy of the step's inputs from "
+                          "pinned memory, scatter of the appended K/V/indexer rows, qsa_forward, D2H copy of the "
+                          "output, stream sync"}
+
+
+ATTN_SETS = {"decode_8k_b1": 16, "decode_64k_b16": 8, "decode_1m_b4": 8}
+
+
+def run_ours(args, wl):
+    env = Env(args)
+    torch, qsa = env.torch, env.qsa
+    hbm_peak, tc_peak, peak_kind = load_peaks()
+
+    B = Bench(env, wl)
+    clocks = Clocks(env.local) if env.rank == 0 else None
     time.sleep(0.3)
-    barrier()
+    env.barrier()
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
-    ms = timed(graph.replay, args.steps)
+    ms_per_step, ms_eager, graph = B.step_timing(args)
     torch.cuda.synchronize()
-    barrier()
+    env.barrier()
     wall = time.perf_counter() - wall0
     clk = clocks.stop() if clocks else None
-    ms_per_step = max_ms(sum(ms) / len(ms))
-    value = job_tokens_per_s(world, n_q_unit, ms_per_step)
-    ms_eager = max_ms(float(np.mean(timed(unit, args.steps))))
-
-    # ---- per-kernel breakdown through the standalone entry points (same inputs) ----
-    T = steps[-1]
-    n_q, mb = T["n_q"], T["max_blocks"]
-    ld = (mb + 3) // 4 * 4
-    scores = torch.empty((n_q, ld), dtype=torch.float32, device="cuda")
-    out_k = torch.empty_like(outs[-1])
-    sel_k, cnt_k = sels[-1].clone(), cnts[-1].clone()
-    ws_k = torch.empty(qsa.qsa_workspace_bytes(dims, n_q, mb, 0), dtype=torch.uint8, device="cuda")
-    qsa.qsa_workspace_init(ws_k)
-    kernels = {}
-    if mode == qsa.QSA_MODE_DECODE:
-        run_score = lambda: qsa.qsa_index_scores(dims, T["q_idx"], T["w"], dw.pooled, T["q_seq"], T["q_pos"], n_q,
-                                                  mb, scores, ld, ws_k)
-        run_score()
-        run_topk = lambda: qsa.qsa_topk_blocks(dims, scores, ld, T["q_pos"], n_q, mb, sel_k, cnt_k, ws_k)
-        run_topk()  # first launch of its kernels outside the timing (module loading)
-        kernels["index_scores_us"] = 1e3 * float(np.mean(timed(run_score, args.steps)))
-        kernels["topk_us"] = 1e3 * float(np.mean(timed(run_topk, args.steps)))
-    run_attn = lambda: qsa.qsa_sparse_attn(dims, T["q"], dw.k_cache, dw.v_cache, T["q_seq"], T["q_pos"], sel_k,
-                                            cnt_k, n_q, out_k, ws_k)
-    run_attn()
-    attn_ms = float(np.mean(timed(run_attn, args.steps)))
-    kernels["sparse_attn_us"] = 1e3 * attn_ms
-    kernels["attn_matches_forward"] = bool(torch.equal(out_k, outs[-1]))
-    kernels["step_eager_us"] = 1e3 * ms_eager
-
-    # algorithmic bytes of the gathered attention: K+V rows of every attended token
-    # (4 per selected block plus the partial block) for every KV head, q in, out written
-    cnt_h = cnt_k.cpu().numpy().astype(np.int64)
-    part = (np.asarray(wl.steps[-1].q_pos, dtype=np.int64) + 1) % wl.block_size
-    toks = cnt_h * wl.block_size + part
-    attn_bytes = int(toks.sum() * wl.n_kv_heads * wl.head_dim * 2 * 2 + 2 * n_q * wl.n_q_heads * wl.head_dim * 2)
-    hbm_peak, tc_peak, peak_kind = load_peaks()
-    achieved = attn_bytes / (attn_ms / 1e3) / 1e9
-    roofline = {"kernel": "k_sparse_attn", "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
-                "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
-                "peak_source": f"{peak_kind} hbm_gbs (burst copy)",
-                "algorithmic_bytes_per_launch": attn_bytes, "traffic": load_traffic("k_sparse_attn", wl.name)}
-
-    # ---- end to end: host buffers in, host buffer out, copies inside the timed region ----
-    # Every step's inputs travel in one pinned host buffer: queries, indexer inputs,
-    # positions, and the appended tokens' K/V rows and indexer keys, which are
-    # scattered into the caches on the device.
-    e2e_steps = []
-    for si, T in enumerate(steps):
-        st = wl.steps[si]
-        parts = {k: T[k] for k in ("q", "q_idx", "w", "len_before", "len_after", "q_seq", "q_pos")}
-        new = [(s, a, b) for s, (a, b) in enumerate(zip(st.len_before, st.len_after)) if b > a]
-        seq_i = torch.tensor([s for s, a, b in new for _ in range(a, b)], dtype=torch.int64, device="cuda")
-        pos_i = torch.tensor([p for s, a, b in new for p in range(a, b)], dtype=torch.int64, device="cuda")
-        parts["k_new"] = dw.k_cache[seq_i, :, pos_i].contiguous()
-        parts["v_new"] = dw.v_cache[seq_i, :, pos_i].contiguous()
-        parts["ik_new"] = dw.idx_k[seq_i, pos_i].contiguous()
-        layout, off = {}, 0
-        for k, v in parts.items():
-            nb = v.numel() * v.element_size()
-            layout[k] = (off, nb, v.dtype, tuple(v.shape))
-            off += (nb + 255) // 256 * 256
-        h_in = torch.empty(off, dtype=torch.uint8).pin_memory()
-        for k, v in parts.items():
-            o, nb, _, _ = layout[k]
-            h_in[o:o + nb].copy_(v.reshape(-1).view(torch.uint8).cpu())
-        d_in = torch.empty(off, dtype=torch.uint8, device="cuda")
-        view = {k: d_in[o:o + nb].view(dt).view(shape) for k, (o, nb, dt, shape) in layout.items()}
-        h_out = torch.empty(tuple(outs[si].shape), dtype=outs[si].dtype).pin_memory()
-        e2e_steps.append((T, h_in, d_in, view, seq_i, pos_i, h_out))
-
-    def unit_e2e():
-        for (T, h_in, d_in, view, seq_i, pos_i, h_out), out, sel, cnt in zip(e2e_steps, outs, sels, cnts):
-            d_in.copy_(h_in, non_blocking=True)
-            dw.k_cache[seq_i, :, pos_i] = view["k_new"]
-            dw.v_cache[seq_i, :, pos_i] = view["v_new"]
-            dw.idx_k[seq_i, pos_i] = view["ik_new"]
-            forward(T, out, sel, cnt, src=view)
-            h_out.copy_(out, non_blocking=True)
-
-    for _ in range(3):
-        unit_e2e()
-    torch.cuda.synchronize()
-    graph_e2e = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_e2e):
-        unit_e2e()
-    e2e_ms = []
-    for _ in range(args.steps):
-        flush()
-        torch.cuda.synchronize()
-        t0 = time.perf_counter()
-        graph_e2e.replay()
-        torch.cuda.current_stream().synchronize()
-        e2e_ms.append(1e3 * (time.perf_counter() - t0))
-    e2e_ms = max_ms(float(np.mean(e2e_ms)))
-    h2d = sum(x[1].numel() for x in e2e_steps)
-    d2h = sum(x[6].numel() * x[6].element_size() for x in e2e_steps)
-    e2e = {"value": job_tokens_per_s(world, n_q_unit, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
-           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-           "timing": "host wall clock around one CUDA-graph replay of: one H2D copy of the step's inputs from "
-                     "pinned memory, scatter of the appended K/V/indexer rows, qsa_forward, D2H copy of the "
-                     "output, stream sync"}
-
-    flags = qsa.qsa_read_device_status(ws)
-    launches_per_step = sum(forward_launches(wl, mode == qsa.QSA_MODE_PREFILL, T) for T in steps)
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+    value = job_tokens_per_s(env.world, B.n_q_unit, ms_per_step)
+    del graph
+    kern = B.kernels(args, hbm_peak, tc_peak, peak_kind, ATTN_SETS.get(wl.name, 4))
+    kern["step_eager_us"] = 1e3 * ms_eager
+    e2e = B.e2e(args)
+    flags = qsa.qsa_read_device_status(B.ws)
+    roofline = dict(kern["roofline_attention"])
+    roofline["traffic"] = load_traffic(roofline["kernel"], wl.name)
+    launches_per_step = sum(forward_launches(wl, B.mode == qsa.QSA_MODE_PREFILL, T) for T in B.steps)
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": env.world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded SplitMix64 inputs, integer indexer inputs, approx. N(0,1) Q/K/V)",
-            "config": dict(workload_config(wl), parallelism=f"replicas x{world} (independent sequences per GPU)",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded SplitMix64 inputs, integer indexer inputs, approx. N(0,1) Q/K/V)",
+            "config": dict(workload_config(wl), parallelism=f"replicas x{env.world} (independent sequences per GPU)",
                            execution="CUDA graph of the unit's qsa_forward calls"),
-            "roofline": roofline, "kernels": kernels, "e2e": e2e,
+            "roofline": roofline, "roofline_select": kern["roofline_select"],
+            "kernels": {k: v for k, v in kern.items() if not k.startswith("roofline")}, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clk,
             "wall_s_timed_region": round(wall, 4), "device_status": flags}
-    if rank == 0 and not args.no_cpu_baseline:
+    if env.rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
-    if rank == 0:
+    del B
+    torch.cuda.empty_cache()
+
+    # every other synthetic configuration: its own step time, throughput and rooflines
+    if args.workload_map and env.world == 1:
+        from qsa_synth import workloads as W
+        wmap = {}
+        for f in W.ALL:
+            other = f()
+            if other.name == wl.name:
+                continue
+            Bo = Bench(env, other)
+            steps = max(3, min(args.steps, 5)) if other.mode == "prefill" else args.steps
+            a2 = argparse.Namespace(**dict(vars(args), steps=steps))
+            ms, _, g = Bo.step_timing(a2)
+            del g
+            k2 = Bo.kernels(a2, hbm_peak, tc_peak, peak_kind, ATTN_SETS.get(other.name, 4))
+            wmap[other.name] = {"tokens_per_s": job_tokens_per_s(1, Bo.n_q_unit, ms), "ms_per_unit": ms,
+                                "queries_per_unit": Bo.n_q_unit, "steps_timed": steps,
+                                "select_us": k2["select_us"], "attn_us": k2["attn_us"],
+                                "roofline_select": k2["roofline_select"],
+                                "roofline_attention": k2["roofline_attention"],
+                                "device_status": qsa.qsa_read_device_status(Bo.ws)}
+            del Bo
+            torch.cuda.empty_cache()
+        line["workloads"] = wmap
+        line["workloads_note"] = ("each configuration measured alone on this GPU after the headline: CUDA-graph "
+                                  "replays of its whole unit with L2 flushed before each; selection and attention "
+                                  "timed through their standalone entry points")
+    if env.rank == 0:
         print(json.dumps(line), flush=True)
-    del graph, graph_e2e
-    if world > 1:
-        dist.destroy_process_group()
+    if env.world > 1:
+        env.dist.destroy_process_group()
 
 
 def main():

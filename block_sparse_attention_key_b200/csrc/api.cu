@@ -26,8 +26,12 @@ int check_dims(const qsa_dims* d)
     if (!d) return QSA_ERR_INVALID_ARG;
     if (d->batch < 1 || d->n_q_heads < 1 || d->n_kv_heads < 1) return QSA_ERR_INVALID_ARG;
     if (d->n_q_heads % d->n_kv_heads != 0) return QSA_ERR_INVALID_ARG;
-    if (d->block_size != kBlock || d->top_k != kTopK) return QSA_ERR_INVALID_ARG;
-    if (d->kv_capacity <= 0 || d->kv_capacity % kBlock != 0 || d->kv_capacity >= (1ll << 31))
+    // block size: a power of two up to 16 (4 in the published setting, 1 for per-token
+    // selection); top_k: 1 .. 512 blocks (512 published)
+    if (d->block_size < 1 || d->block_size > kMaxBlockSize || (d->block_size & (d->block_size - 1)) != 0)
+        return QSA_ERR_INVALID_ARG;
+    if (d->top_k < 1 || d->top_k > kSelCap) return QSA_ERR_INVALID_ARG;
+    if (d->kv_capacity <= 0 || d->kv_capacity % d->block_size != 0 || d->kv_capacity >= (1ll << 31))
         return QSA_ERR_INVALID_ARG;
     if (!std::isfinite(d->softmax_scale)) return QSA_ERR_INVALID_ARG;
     if (d->head_dim != kHeadDim || d->n_idx_heads != kIdxHeads || d->idx_dim != kIdxDim)
@@ -38,8 +42,24 @@ int check_dims(const qsa_dims* d)
 
 int check_rows(const qsa_dims* d, int32_t n_q, int64_t max_blocks)
 {
-    if (n_q < 0 || max_blocks < 0 || max_blocks > d->kv_capacity / kBlock) return QSA_ERR_INVALID_ARG;
+    if (n_q < 0 || max_blocks < 0 || max_blocks > d->kv_capacity / d->block_size) return QSA_ERR_INVALID_ARG;
     if (n_q > 65535) return QSA_ERR_UNSUPPORTED;
+    return QSA_OK;
+}
+
+int check_groups(const qsa_dims* d, int32_t n_q, int32_t group_q)
+{
+    if (group_q < 1 || n_q % group_q != 0) return QSA_ERR_INVALID_ARG;
+    if ((int64_t)group_q * (d->n_q_heads / d->n_kv_heads) > 32) return QSA_ERR_UNSUPPORTED;
+    return QSA_OK;
+}
+
+int check_pages(const qsa_dims* d, const int32_t* page_table, int32_t page_tokens, int64_t n_pages)
+{
+    if (!page_table) return QSA_OK;
+    if (!aligned16(page_table) || page_tokens < 1 || page_tokens % d->block_size != 0 ||
+        d->kv_capacity % page_tokens != 0 || n_pages < 1 || n_pages > (1ll << 31) - 1)
+        return QSA_ERR_INVALID_ARG;
     return QSA_OK;
 }
 
@@ -67,7 +87,6 @@ WsLayout plan_workspace(const qsa_dims& d, int32_t n_q, int64_t max_blocks, int3
     L.score_rows = rows;
     L.chunk = select_chunk(max_blocks, rows);
     L.n_chunks = max_blocks > 0 ? (int)((max_blocks + L.chunk - 1) / L.chunk) : 0;
-    L.n_split = mode == QSA_MODE_PREFILL ? 1 : attn_splits(n_q, d.n_kv_heads);
 
     // zeroed region: attention split counters, then the select control blocks
     L.attn_cnt = off;
@@ -77,14 +96,15 @@ WsLayout plan_workspace(const qsa_dims& d, int32_t n_q, int64_t max_blocks, int3
     L.cand = off;
     off += align_up((size_t)rows * kCandCap * 8);
     L.tmp = off;
-    off += align_up((size_t)rows * kTopK * 4);
+    off += align_up((size_t)rows * kSelCap * 4);
     L.score_ld = (max_blocks + 3) / 4 * 4;
     L.scores = off;
     off += align_up((size_t)rows * L.score_ld * 4);
     L.sel = off;
-    off += align_up((size_t)n_q * kTopK * 4 + (size_t)n_q * 4);
+    off += align_up((size_t)n_q * kSelCap * 4 + (size_t)n_q * 4);
+    // decode attention partials, for a merge of split CTAs through global memory
     L.partial = off;
-    if (L.n_split > 1) off += align_up((size_t)n_q * d.n_kv_heads * L.n_split * (32 + 16 * kHeadDim) * 4);
+    if (n_q > 0) off += align_up(attn_decode_partial_bytes());
     if (mode == QSA_MODE_PREFILL && max_blocks > 0 && n_q > 0) {
         L.pf_split = prefill_splits(n_q, max_blocks);
         const size_t segs = (size_t)n_q * 2 * L.pf_split;
@@ -102,8 +122,103 @@ WsLayout plan_workspace(const qsa_dims& d, int32_t n_q, int64_t max_blocks, int3
         L.pf_scratch = off;
         off += align_up((size_t)L.pf_fb_ctas * max_blocks * 4);
     }
+    L.qpos_loc = off;
+    off += align_up((size_t)n_q * 4);
     L.total = off;
     return L;
+}
+
+// Gathered attention for one call.  Calls with many (query, KV head) pairs, dense
+// caches and one query per selection (prefill chunks, large decode batches) run
+// k_sparse_attn, one CTA per pair at two CTAs per SM; everything else (few pairs:
+// splits over the block list; draft-query groups; paged caches) runs k_attn_decode.
+static cudaError_t run_attention(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,
+                                 const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,
+                                 const int32_t* sel_cnt, const int32_t* page_table, int32_t page_tokens,
+                                 int64_t n_pages, int32_t n_q, int32_t group_q, void* out, const WsLayout& L,
+                                 char* ws, cudaStream_t st, bool pdl, bool counters_zeroed)
+{
+    const int64_t n_groups = n_q / group_q;
+    const int64_t pairs = n_groups * d.n_kv_heads;
+    float* partial = (float*)(ws + L.partial);
+    unsigned* counters = (unsigned*)(ws + L.attn_cnt);
+    if (!page_table && group_q == 1 && pairs >= 2 * 148)
+        return launch_attention(d, q, k_cache, v_cache, q_seq, q_pos, sel_idx, sel_cnt, n_q, out, 1, partial,
+                                counters, (unsigned*)ws, st, pdl);
+    return launch_attn_decode(d, q, k_cache, v_cache, q_seq, q_pos, sel_idx, sel_cnt, page_table, page_tokens,
+                              n_pages, n_groups, group_q, out, partial, counters, (unsigned*)ws, st, pdl, true,
+                              counters_zeroed);
+}
+
+// Steps 2 + 3 for `n_rows` selection rows (one per group of group_q queries) into
+// sel_idx / sel_cnt.  Decode rows expect their control blocks zeroed already.
+static cudaError_t run_select(const qsa_dims& d, const void* q_idx, const float* w, const void* pooled,
+                              const int32_t* q_seq, const int32_t* q_pos, int32_t n_rows, int32_t group_q,
+                              int64_t max_blocks, int32_t mode, int32_t* sel_idx, int32_t* sel_cnt,
+                              const WsLayout& L, char* ws, unsigned* status, cudaStream_t st, bool pdl)
+{
+    cudaError_t e = cudaSuccess;
+    if (max_blocks == 0) {
+        e = cudaMemsetAsync(sel_idx, 0xFF, (size_t)n_rows * kSelCap * 4, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(sel_cnt, 0, (size_t)n_rows * 4, st);
+        return e;
+    }
+    if (mode == QSA_MODE_DECODE) {
+        TopkCtrl* ctrl = (TopkCtrl*)(ws + L.ctrl);
+        float* scores = (float*)(ws + L.scores);
+        // rows of up to 16,384 blocks are selected by the scoring kernel's last CTA per row
+        const bool in_kernel = max_blocks <= kScoreFinishMaxBlocks;
+        e = launch_score_decode(d, q_idx, w, pooled, q_seq, q_pos, 0, n_rows, max_blocks, scores, L.score_ld,
+                                L.chunk, ctrl, in_kernel ? sel_idx : nullptr, in_kernel ? sel_cnt : nullptr, status,
+                                st, pdl, group_q);
+        if (e != cudaSuccess || in_kernel) return e;
+        return launch_topk(scores, L.score_ld, q_pos, 0, n_rows, max_blocks, d.kv_capacity, d.block_size, d.top_k,
+                           L.chunk, L.n_chunks, ctrl, (unsigned long long*)(ws + L.cand), (int32_t*)(ws + L.tmp), sel_idx, sel_cnt, true,
+                           status, st, pdl);
+    }
+    // prefill chunk: tensor-core scoring with streaming admission
+    e = cudaMemsetAsync(ws + L.pf_theta, 0, (size_t)(n_rows + 1) * 4, st);
+    if (e != cudaSuccess) return e;
+    return launch_prefill_select(d, q_idx, w, pooled, q_seq, q_pos, n_rows, max_blocks, L.pf_split,
+                                 (unsigned long long*)(ws + L.pf_cand), (unsigned*)(ws + L.pf_cnt),
+                                 (unsigned*)(ws + L.pf_theta), (uint32_t*)(ws + L.pf_shist),
+                                 (int32_t*)(ws + L.pf_work), (float*)(ws + L.pf_scratch), L.pf_fb_ctas, sel_idx,
+                                 sel_cnt, status, st);
+}
+
+// A serving batch in one call: rows [0, n_decode) are decode queries (any sequences,
+// scored through score rows), rows [n_decode, n_q) are prefill chunks (tensor-core
+// scoring); one pooling launch before and one attention launch over every row after.
+// The workspace holds a decode layout, then a prefill layout; the status word is the
+// first one's.
+static int forward_mixed(const qsa_dims& d, const qsa_forward_args& a, char* ws, size_t ws_bytes, cudaStream_t st)
+{
+    const int32_t n_q = a.n_q, n_dec = a.n_decode, n_pf = n_q - n_dec;
+    const WsLayout Ld = plan_workspace(d, n_q, a.max_blocks, QSA_MODE_DECODE);
+    const WsLayout Lp = plan_workspace(d, n_q, a.max_blocks, QSA_MODE_PREFILL);
+    if (ws_bytes < Ld.total + Lp.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
+    unsigned* status = (unsigned*)ws;
+    int32_t* sel_idx = a.sel_idx ? a.sel_idx : (int32_t*)(ws + Ld.sel);
+    int32_t* sel_cnt = a.sel_cnt ? a.sel_cnt : (int32_t*)(ws + Ld.sel) + (size_t)n_q * kSelCap;
+    // pool the appended blocks; the same launch clears the decode rows' control blocks
+    cudaError_t e = launch_pool(d, a.idx_k, a.pooled, a.len_before, a.len_after, a.max_new_tokens, ws + Ld.attn_cnt,
+                                Ld.ctrl_bytes, status, st);
+    if (e != cudaSuccess) return QSA_ERR_CUDA;
+    if (n_dec > 0) {
+        e = run_select(d, a.q_idx, a.w, a.pooled, a.q_seq, a.q_pos, n_dec, 1, a.max_blocks, QSA_MODE_DECODE, sel_idx,
+                       sel_cnt, Ld, ws, status, st, false);
+        if (e != cudaSuccess) return QSA_ERR_CUDA;
+    }
+    if (n_pf > 0) {
+        const size_t qrow = (size_t)kIdxHeads * kIdxDim * 2;
+        e = run_select(d, (const char*)a.q_idx + (size_t)n_dec * qrow, a.w + (size_t)n_dec * kIdxHeads, a.pooled,
+                       a.q_seq + n_dec, a.q_pos + n_dec, n_pf, 1, a.max_blocks, QSA_MODE_PREFILL,
+                       sel_idx + (size_t)n_dec * kSelCap, sel_cnt + n_dec, Lp, ws + Ld.total, status, st, false);
+        if (e != cudaSuccess) return QSA_ERR_CUDA;
+    }
+    if (n_q == 0) return QSA_OK;
+    return cuda_status(run_attention(d, a.q, a.k_cache, a.v_cache, a.q_seq, a.q_pos, sel_idx, sel_cnt, a.page_table,
+                                     a.page_tokens, a.n_pages, n_q, 1, a.out, Ld, ws, st, false, true));
 }
 
 }  // namespace qsa
@@ -115,6 +230,9 @@ extern "C" {
 size_t qsa_workspace_bytes(const qsa_dims* dims, int32_t n_q, int64_t max_blocks, int32_t mode)
 {
     if (check_dims(dims) != QSA_OK || check_rows(dims, n_q, max_blocks) != QSA_OK) return 0;
+    if (mode == QSA_MODE_MIXED)
+        return plan_workspace(*dims, n_q, max_blocks, QSA_MODE_DECODE).total +
+               plan_workspace(*dims, n_q, max_blocks, QSA_MODE_PREFILL).total;
     if (mode != QSA_MODE_DECODE && mode != QSA_MODE_PREFILL) return 0;
     return plan_workspace(*dims, n_q, max_blocks, mode).total;
 }
@@ -122,7 +240,9 @@ size_t qsa_workspace_bytes(const qsa_dims* dims, int32_t n_q, int64_t max_blocks
 int qsa_workspace_init(void* workspace, size_t ws_bytes, void* stream)
 {
     if (!aligned16(workspace) || ws_bytes < kAlign) return QSA_ERR_INVALID_ARG;
-    return cuda_status(cudaMemsetAsync(workspace, 0, kAlign, (cudaStream_t)stream));
+    // the status word and every completion counter start at zero (counters return to
+    // zero at the end of every launch that uses them)
+    return cuda_status(cudaMemsetAsync(workspace, 0, ws_bytes, (cudaStream_t)stream));
 }
 
 int qsa_read_device_status(void* workspace, uint32_t* flags, void* stream)
@@ -200,14 +320,14 @@ int qsa_topk_blocks(const qsa_dims* dims, const float* scores, int64_t ld_scores
     char* ws = (char*)workspace;
     if (max_blocks == 0) {
         // no candidates at all: empty selections
-        cudaError_t e = cudaMemsetAsync(sel_idx, 0xFF, (size_t)n_q * kTopK * 4, st);
+        cudaError_t e = cudaMemsetAsync(sel_idx, 0xFF, (size_t)n_q * kSelCap * 4, st);
         if (e == cudaSuccess) e = cudaMemsetAsync(sel_cnt, 0, (size_t)n_q * 4, st);
         return cuda_status(e);
     }
     cudaError_t e = cudaMemsetAsync(ws + L.attn_cnt, 0, L.ctrl_bytes, st);
     if (e != cudaSuccess) return QSA_ERR_CUDA;
-    return cuda_status(launch_topk(scores, ld_scores, q_pos, 0, n_q, max_blocks, dims->kv_capacity, L.chunk,
-                                   L.n_chunks, (TopkCtrl*)(ws + L.ctrl), (unsigned long long*)(ws + L.cand),
+    return cuda_status(launch_topk(scores, ld_scores, q_pos, 0, n_q, max_blocks, dims->kv_capacity,
+                                   dims->block_size, dims->top_k, L.chunk, L.n_chunks, (TopkCtrl*)(ws + L.ctrl), (unsigned long long*)(ws + L.cand),
                                    (int32_t*)(ws + L.tmp), sel_idx, sel_cnt, false, (unsigned*)ws, st));
 }
 
@@ -215,24 +335,63 @@ int qsa_sparse_attn(const qsa_dims* dims, const void* q, const void* k_cache, co
                     const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx, const int32_t* sel_cnt,
                     int32_t n_q, void* out, void* workspace, size_t ws_bytes, void* stream)
 {
+    qsa_attn_args a = {};
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.q_seq = q_seq;
+    a.q_pos = q_pos;
+    a.sel_idx = sel_idx;
+    a.sel_cnt = sel_cnt;
+    a.n_q = n_q;
+    a.group_q = 1;
+    a.out = out;
+    return qsa_sparse_attn_ex(dims, &a, workspace, ws_bytes, stream);
+}
+
+int qsa_sparse_attn_ex(const qsa_dims* dims, const qsa_attn_args* a, void* workspace, size_t ws_bytes, void* stream)
+{
     int rc = check_dims(dims);
     if (rc != QSA_OK) return rc;
-    if ((rc = check_rows(dims, n_q, 0)) != QSA_OK) return rc;
-    if (n_q == 0) return QSA_OK;
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(q_seq) || !aligned16(q_pos) ||
-        !aligned16(sel_idx) || !aligned16(sel_cnt) || !aligned16(out) || !aligned16(workspace))
+    if (!a) return QSA_ERR_INVALID_ARG;
+    if ((rc = check_rows(dims, a->n_q, 0)) != QSA_OK) return rc;
+    if ((rc = check_groups(dims, a->n_q, a->group_q < 1 ? 0 : a->group_q)) != QSA_OK) return rc;
+    if ((rc = check_pages(dims, a->page_table, a->page_tokens, a->n_pages)) != QSA_OK) return rc;
+    if (a->n_q == 0) return QSA_OK;
+    if (!aligned16(a->q) || !aligned16(a->k_cache) || !aligned16(a->v_cache) || !aligned16(a->q_seq) ||
+        !aligned16(a->q_pos) || !aligned16(a->sel_idx) || !aligned16(a->sel_cnt) || !aligned16(a->out) ||
+        !aligned16(workspace))
         return QSA_ERR_INVALID_ARG;
-    const WsLayout L = plan_workspace(*dims, n_q, 0, QSA_MODE_DECODE);
+    const WsLayout L = plan_workspace(*dims, a->n_q, 0, QSA_MODE_DECODE);
+    if (ws_bytes < L.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
+    // split counters: zero since qsa_workspace_init, and every merge resets its own
+    return cuda_status(run_attention(*dims, a->q, a->k_cache, a->v_cache, a->q_seq, a->q_pos, a->sel_idx, a->sel_cnt,
+                                     a->page_table, a->page_tokens, a->n_pages, a->n_q, a->group_q, a->out, L,
+                                     (char*)workspace, (cudaStream_t)stream, false, true));
+}
+
+int qsa_select_blocks(const qsa_dims* dims, const void* q_idx, const float* w, const void* pooled,
+                      const int32_t* q_seq, const int32_t* q_pos, int32_t n_q, int64_t max_blocks, int32_t mode,
+                      int32_t* sel_idx, int32_t* sel_cnt, void* workspace, size_t ws_bytes, void* stream)
+{
+    int rc = check_dims(dims);
+    if (rc != QSA_OK) return rc;
+    if ((rc = check_rows(dims, n_q, max_blocks)) != QSA_OK) return rc;
+    if (mode != QSA_MODE_DECODE && mode != QSA_MODE_PREFILL) return QSA_ERR_INVALID_ARG;
+    if (n_q == 0) return QSA_OK;
+    if (!aligned16(q_idx) || !aligned16(w) || !aligned16(pooled) || !aligned16(q_seq) || !aligned16(q_pos) ||
+        !aligned16(sel_idx) || !aligned16(sel_cnt) || !aligned16(workspace))
+        return QSA_ERR_INVALID_ARG;
+    const WsLayout L = plan_workspace(*dims, n_q, max_blocks, mode);
     if (ws_bytes < L.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t st = (cudaStream_t)stream;
     char* ws = (char*)workspace;
-    if (L.n_split > 1) {
-        cudaError_t e = cudaMemsetAsync(ws + L.attn_cnt, 0, (size_t)n_q * dims->n_kv_heads * 4, st);
+    if (mode == QSA_MODE_DECODE && max_blocks > 0) {
+        const cudaError_t e = cudaMemsetAsync(ws + L.ctrl, 0, (size_t)n_q * sizeof(TopkCtrl), st);
         if (e != cudaSuccess) return QSA_ERR_CUDA;
     }
-    return cuda_status(launch_attention(*dims, q, k_cache, v_cache, q_seq, q_pos, sel_idx, sel_cnt, n_q, out,
-                                        L.n_split, (float*)(ws + L.partial), (unsigned*)(ws + L.attn_cnt),
-                                        (unsigned*)ws, st));
+    return cuda_status(run_select(*dims, q_idx, w, pooled, q_seq, q_pos, n_q, 1, max_blocks, mode, sel_idx, sel_cnt,
+                                  L, ws, (unsigned*)ws, st, false));
 }
 
 int qsa_forward(const qsa_dims* dims, const qsa_forward_args* a, void* workspace, size_t ws_bytes, void* stream)
@@ -241,7 +400,13 @@ int qsa_forward(const qsa_dims* dims, const qsa_forward_args* a, void* workspace
     if (rc != QSA_OK) return rc;
     if (!a) return QSA_ERR_INVALID_ARG;
     if ((rc = check_rows(dims, a->n_q, a->max_blocks)) != QSA_OK) return rc;
-    if (a->mode != QSA_MODE_DECODE && a->mode != QSA_MODE_PREFILL) return QSA_ERR_INVALID_ARG;
+    if (a->mode != QSA_MODE_DECODE && a->mode != QSA_MODE_PREFILL && a->mode != QSA_MODE_MIXED)
+        return QSA_ERR_INVALID_ARG;
+    if (a->mode == QSA_MODE_MIXED && (a->n_decode < 0 || a->n_decode > a->n_q)) return QSA_ERR_INVALID_ARG;
+    const int32_t group_q = a->group_q < 1 ? 1 : a->group_q;
+    if (group_q > 1 && a->mode != QSA_MODE_DECODE) return QSA_ERR_INVALID_ARG;
+    if ((rc = check_groups(dims, a->n_q, group_q)) != QSA_OK) return rc;
+    if ((rc = check_pages(dims, a->page_table, a->page_tokens, a->n_pages)) != QSA_OK) return rc;
     if (a->max_new_tokens < 0 || (int64_t)a->max_new_tokens > dims->kv_capacity) return QSA_ERR_INVALID_ARG;
     if (!aligned16(a->idx_k) || !aligned16(a->pooled) || !aligned16(a->len_before) || !aligned16(a->len_after) ||
         !aligned16(workspace))
@@ -253,6 +418,8 @@ int qsa_forward(const qsa_dims* dims, const qsa_forward_args* a, void* workspace
     if ((a->sel_idx && !aligned16(a->sel_idx)) || (a->sel_cnt && !aligned16(a->sel_cnt)))
         return QSA_ERR_INVALID_ARG;
     const int32_t n_q = a->n_q;
+    const int32_t n_groups = n_q / group_q;  // selection rows
+    if (a->mode == QSA_MODE_MIXED) return forward_mixed(*dims, *a, (char*)workspace, ws_bytes, (cudaStream_t)stream);
     const WsLayout L = plan_workspace(*dims, n_q, a->max_blocks, a->mode);
     if (ws_bytes < L.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
 
@@ -261,32 +428,21 @@ int qsa_forward(const qsa_dims* dims, const qsa_forward_args* a, void* workspace
     unsigned* status = (unsigned*)ws;
     cudaError_t e = cudaSuccess;
     int32_t* sel_idx = a->sel_idx ? a->sel_idx : (int32_t*)(ws + L.sel);
-    int32_t* sel_cnt = a->sel_cnt ? a->sel_cnt : (int32_t*)(ws + L.sel) + (size_t)n_q * kTopK;
-
+    int32_t* sel_cnt = a->sel_cnt ? a->sel_cnt : (int32_t*)(ws + L.sel) + (size_t)n_q * kSelCap;
     if (n_q > 0 && a->max_blocks > 0 && a->mode == QSA_MODE_DECODE) {
         // decode chain, each kernel launched as a programmatic dependent of the one
         // before: pool (+ clearing of the split counters and select control blocks),
-        // scores with the digit-1 histogram, select, attention
+        // scores with the digit-1 histogram, select, attention; one selection row per
+        // group of draft queries, scored at the group's first query
         e = launch_pool(*dims, a->idx_k, a->pooled, a->len_before, a->len_after, a->max_new_tokens, ws + L.attn_cnt,
                         L.ctrl_bytes, status, st);
         if (e != cudaSuccess) return QSA_ERR_CUDA;
-        TopkCtrl* ctrl = (TopkCtrl*)(ws + L.ctrl);
-        float* scores = (float*)(ws + L.scores);
-        // rows of up to 16,384 blocks are selected by the scoring kernel's last CTA per row
-        const bool in_kernel = a->max_blocks <= kScoreFinishMaxBlocks;
-        e = launch_score_decode(*dims, a->q_idx, a->w, a->pooled, a->q_seq, a->q_pos, 0, n_q, a->max_blocks, scores,
-                                L.score_ld, L.chunk, ctrl, in_kernel ? sel_idx : nullptr,
-                                in_kernel ? sel_cnt : nullptr, status, st, true);
+        e = run_select(*dims, a->q_idx, a->w, a->pooled, a->q_seq, a->q_pos, n_groups, group_q, a->max_blocks,
+                       QSA_MODE_DECODE, sel_idx, sel_cnt, L, ws, status, st, true);
         if (e != cudaSuccess) return QSA_ERR_CUDA;
-        if (!in_kernel) {
-            e = launch_topk(scores, L.score_ld, a->q_pos, 0, n_q, a->max_blocks, dims->kv_capacity, L.chunk,
-                            L.n_chunks, ctrl, (unsigned long long*)(ws + L.cand), (int32_t*)(ws + L.tmp), sel_idx,
-                            sel_cnt, true, status, st, true);
-            if (e != cudaSuccess) return QSA_ERR_CUDA;
-        }
-        return cuda_status(launch_attention(*dims, a->q, a->k_cache, a->v_cache, a->q_seq, a->q_pos, sel_idx,
-                                            sel_cnt, n_q, a->out, L.n_split, (float*)(ws + L.partial),
-                                            (unsigned*)(ws + L.attn_cnt), status, st, true));
+        return cuda_status(run_attention(*dims, a->q, a->k_cache, a->v_cache, a->q_seq, a->q_pos, sel_idx, sel_cnt,
+                                         a->page_table, a->page_tokens, a->n_pages, n_q, group_q, a->out, L, ws, st,
+                                         true, true));
     }
 
     if (a->max_new_tokens > 0) {
@@ -296,27 +452,114 @@ int qsa_forward(const qsa_dims* dims, const qsa_forward_args* a, void* workspace
     }
     if (n_q == 0) return QSA_OK;
 
-    if (a->max_blocks == 0) {
-        e = cudaMemsetAsync(sel_idx, 0xFF, (size_t)n_q * kTopK * 4, st);
-        if (e == cudaSuccess) e = cudaMemsetAsync(sel_cnt, 0, (size_t)n_q * 4, st);
-        if (e != cudaSuccess) return QSA_ERR_CUDA;
-    } else {
-        // prefill chunk: tensor-core scoring with streaming admission
-        e = cudaMemsetAsync(ws + L.pf_theta, 0, (size_t)(n_q + 1) * 4, st);
-        if (e != cudaSuccess) return QSA_ERR_CUDA;
-        e = launch_prefill_select(*dims, a->q_idx, a->w, a->pooled, a->q_seq, a->q_pos, n_q, a->max_blocks,
-                                  L.pf_split, (unsigned long long*)(ws + L.pf_cand), (unsigned*)(ws + L.pf_cnt),
-                                  (unsigned*)(ws + L.pf_theta), (uint32_t*)(ws + L.pf_shist), (int32_t*)(ws + L.pf_work),
-                                  (float*)(ws + L.pf_scratch), L.pf_fb_ctas, sel_idx, sel_cnt, status, st);
-        if (e != cudaSuccess) return QSA_ERR_CUDA;
-    }
-    if (L.n_split > 1) {
-        e = cudaMemsetAsync(ws + L.attn_cnt, 0, (size_t)n_q * dims->n_kv_heads * 4, st);
-        if (e != cudaSuccess) return QSA_ERR_CUDA;
-    }
-    return cuda_status(launch_attention(*dims, a->q, a->k_cache, a->v_cache, a->q_seq, a->q_pos, sel_idx, sel_cnt,
-                                        n_q, a->out, L.n_split, (float*)(ws + L.partial),
-                                        (unsigned*)(ws + L.attn_cnt), status, st));
+    // a prefill chunk (or a decode call with no complete block anywhere)
+    e = run_select(*dims, a->q_idx, a->w, a->pooled, a->q_seq, a->q_pos, n_groups, group_q, a->max_blocks,
+                   QSA_MODE_PREFILL, sel_idx, sel_cnt, L, ws, status, st, false);
+    if (e != cudaSuccess) return QSA_ERR_CUDA;
+    return cuda_status(run_attention(*dims, a->q, a->k_cache, a->v_cache, a->q_seq, a->q_pos, sel_idx, sel_cnt,
+                                     a->page_table, a->page_tokens, a->n_pages, n_q, group_q, a->out, L, ws, st, false,
+                                     true));
+}
+
+// ---------------------------------------------------------------- context parallelism
+
+static int check_shard(const qsa_dims* shard, int32_t n_q, int64_t blk_lo)
+{
+    int rc = check_dims(shard);
+    if (rc != QSA_OK) return rc;
+    if ((rc = check_rows(shard, n_q, 0)) != QSA_OK) return rc;
+    if (blk_lo < 0 || (blk_lo + shard->kv_capacity / shard->block_size) * shard->block_size >= (1ll << 31))
+        return QSA_ERR_INVALID_ARG;
+    return QSA_OK;
+}
+
+size_t qsa_cp_workspace_bytes(const qsa_dims* shard, int32_t n_q)
+{
+    if (check_shard(shard, n_q, 0) != QSA_OK) return 0;
+    return plan_workspace(*shard, n_q, shard->kv_capacity / shard->block_size, QSA_MODE_DECODE).total;
+}
+
+int qsa_cp_select_keys(const qsa_dims* shard, const void* q_idx, const float* w, const void* pooled_shard,
+                       const int32_t* q_seq, const int32_t* q_pos, int32_t n_q, int64_t blk_lo, uint64_t* keys,
+                       int32_t* key_cnt, void* workspace, size_t ws_bytes, void* stream)
+{
+    int rc = check_shard(shard, n_q, blk_lo);
+    if (rc != QSA_OK) return rc;
+    if (n_q == 0) return QSA_OK;
+    if (!aligned16(q_idx) || !aligned16(w) || !aligned16(pooled_shard) || !aligned16(q_seq) || !aligned16(q_pos) ||
+        !aligned16(keys) || !aligned16(key_cnt) || !aligned16(workspace))
+        return QSA_ERR_INVALID_ARG;
+    const int64_t n_local = shard->kv_capacity / shard->block_size;
+    const WsLayout L = plan_workspace(*shard, n_q, n_local, QSA_MODE_DECODE);
+    if (ws_bytes < L.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t st = (cudaStream_t)stream;
+    char* ws = (char*)workspace;
+    int32_t* pos_loc = (int32_t*)(ws + L.qpos_loc);
+    int32_t* sel = (int32_t*)(ws + L.sel);
+    int32_t* cnt = sel + (size_t)n_q * kSelCap;
+    // positions outside the shard are expected here: their flags go to a word nobody reads
+    unsigned* quiet = (unsigned*)ws + 1;
+    cudaError_t e = launch_cp_local_pos(q_pos, n_q, blk_lo * shard->block_size, shard->kv_capacity, pos_loc, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.ctrl, 0, (size_t)n_q * sizeof(TopkCtrl), st);
+    if (e == cudaSuccess)
+        e = run_select(*shard, q_idx, w, pooled_shard, q_seq, pos_loc, n_q, 1, n_local, QSA_MODE_DECODE, sel, cnt, L, ws,
+                       quiet, st, false);
+    if (e == cudaSuccess)
+        e = launch_cp_keys((const float*)(ws + L.scores), L.score_ld, sel, cnt, n_q, blk_lo,
+                           (unsigned long long*)keys, key_cnt, st);
+    return cuda_status(e);
+}
+
+int qsa_cp_merge_keys(const qsa_dims* shard, int32_t n_ranks, const uint64_t* keys_all, const int32_t* cnt_all,
+                      int32_t n_q, int64_t blk_lo, int32_t* sel_local, int32_t* cnt_local, int32_t* sel_global,
+                      int32_t* cnt_global, void* stream)
+{
+    int rc = check_shard(shard, n_q, blk_lo);
+    if (rc != QSA_OK) return rc;
+    if (n_ranks < 1 || n_ranks > kCandCap / kSelCap) return QSA_ERR_UNSUPPORTED;
+    if (n_q == 0) return QSA_OK;
+    if (!aligned16(keys_all) || !aligned16(cnt_all) || !aligned16(sel_local) || !aligned16(cnt_local) ||
+        (sel_global && !aligned16(sel_global)) || (cnt_global && !aligned16(cnt_global)))
+        return QSA_ERR_INVALID_ARG;
+    return cuda_status(launch_cp_merge((const unsigned long long*)keys_all, cnt_all, n_ranks, n_q, shard->top_k,
+                                       blk_lo, shard->kv_capacity / shard->block_size, sel_local, cnt_local,
+                                       sel_global, cnt_global, (cudaStream_t)stream));
+}
+
+int qsa_cp_attn_partial(const qsa_dims* shard, const void* q, const void* k_shard, const void* v_shard,
+                        const int32_t* q_seq, const int32_t* q_pos, int32_t n_q, int64_t blk_lo,
+                        const int32_t* sel_local, const int32_t* cnt_local, float* part, void* workspace,
+                        size_t ws_bytes, void* stream)
+{
+    int rc = check_shard(shard, n_q, blk_lo);
+    if (rc != QSA_OK) return rc;
+    if (n_q == 0) return QSA_OK;
+    if (!aligned16(q) || !aligned16(k_shard) || !aligned16(v_shard) || !aligned16(q_seq) || !aligned16(q_pos) ||
+        !aligned16(sel_local) || !aligned16(cnt_local) || !aligned16(part) || !aligned16(workspace))
+        return QSA_ERR_INVALID_ARG;
+    const WsLayout L = plan_workspace(*shard, n_q, shard->kv_capacity / shard->block_size, QSA_MODE_DECODE);
+    if (ws_bytes < L.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t st = (cudaStream_t)stream;
+    char* ws = (char*)workspace;
+    int32_t* pos_loc = (int32_t*)(ws + L.qpos_loc);
+    unsigned* quiet = (unsigned*)ws + 1;
+    cudaError_t e = launch_cp_local_pos(q_pos, n_q, blk_lo * shard->block_size, shard->kv_capacity, pos_loc, st);
+    if (e == cudaSuccess)
+        e = launch_attn_decode(*shard, q, k_shard, v_shard, q_seq, pos_loc, sel_local, cnt_local, nullptr, 0, 0, n_q,
+                               1, nullptr, (float*)(ws + L.partial), (unsigned*)(ws + L.attn_cnt), quiet, st, false,
+                               true, true, part);
+    return cuda_status(e);
+}
+
+int qsa_cp_combine(const qsa_dims* dims, int32_t n_ranks, const float* parts_all, int32_t n_q, void* out, void* stream)
+{
+    int rc = check_dims(dims);
+    if (rc != QSA_OK) return rc;
+    if ((rc = check_rows(dims, n_q, 0)) != QSA_OK) return rc;
+    if (n_ranks < 1) return QSA_ERR_INVALID_ARG;
+    if (n_q == 0) return QSA_OK;
+    if (!aligned16(parts_all) || !aligned16(out)) return QSA_ERR_INVALID_ARG;
+    return cuda_status(launch_cp_combine(parts_all, n_ranks, (int64_t)n_q * dims->n_q_heads, out, (cudaStream_t)stream));
 }
 
 }  // extern "C"

@@ -30,13 +30,12 @@ namespace qsa {
 
 namespace {
 
-constexpr int kTileBlocks = 16;
-constexpr int kTileTok = kTileBlocks * kBlock;  // 64 tokens per stage
+constexpr int kTileTok = 64;                     // tokens per stage (64 / block size blocks)
 constexpr int kStages = 3;
 constexpr int kThreads = 128;
 constexpr int kRowBytes = kHeadDim * 2;          // 256 B per token row
 constexpr int kStageBytes = kTileTok * kRowBytes; // 16 KiB of K (or V)
-constexpr int kMaxSplitBlocks = kTopK + 1;        // selected blocks + the partial block
+constexpr int kMaxSplitBlocks = kSelCap + 1;        // selected blocks + the partial block
 constexpr int kMaxClusterSplits = 8;              // splits of one (query, KV head): a portable cluster
 
 constexpr int kSmemQ = 0;
@@ -178,7 +177,8 @@ k_sparse_attn(const uint4* __restrict__ q, const uint16_t* __restrict__ k_cache,
               const uint16_t* __restrict__ v_cache, const int32_t* __restrict__ q_seq,
               const int32_t* __restrict__ q_pos, const int32_t* __restrict__ sel_idx,
               const int32_t* __restrict__ sel_cnt, int batch, int n_q_heads, int n_kv_heads,
-              int64_t kv_capacity, float scale_log2, int blocks_per_split, int n_split, int cluster_merge,
+              int64_t kv_capacity, int bs_log2, int top_k, float scale_log2, int blocks_per_split, int n_split,
+              int cluster_merge,
               __nv_bfloat16* __restrict__ out, float* __restrict__ partial, unsigned* __restrict__ counters,
               unsigned* status)
 {
@@ -196,8 +196,10 @@ k_sparse_attn(const uint4* __restrict__ q, const uint16_t* __restrict__ k_cache,
     const int s = q_seq[i];
     const int t = q_pos[i];
     const bool ok = s >= 0 && s < batch && t >= 0 && (int64_t)t < kv_capacity;
-    const int n_c = ok ? (t + 1) / kBlock : 0;
-    const int n_part = ok ? (t + 1) - kBlock * n_c : 0;  // tokens of the partial block
+    const int bs = 1 << bs_log2;         // tokens per block
+    const int ipt = kTileTok >> bs_log2;  // blocks per stage
+    const int n_c = ok ? (t + 1) >> bs_log2 : 0;
+    const int n_part = ok ? (t + 1) - (n_c << bs_log2) : 0;  // tokens of the partial block
     // query heads of this KV group -> rows 0..G-1 of a 16-row tile, rows >= G zero
     for (int k = tid; k < 16 * 16; k += kThreads) {
         const int row = k >> 4, ch = k & 15;
@@ -211,7 +213,7 @@ k_sparse_attn(const uint4* __restrict__ q, const uint16_t* __restrict__ k_cache,
     if (!ok && split == 0 && g == 0 && tid == 0)
         set_status(status, (s < 0 || s >= batch) ? QSA_DEV_BAD_SEQ : QSA_DEV_BAD_POS);
     int cnt = ok ? sel_cnt[i] : 0;
-    const int cnt_max = n_c < kTopK ? n_c : kTopK;
+    const int cnt_max = n_c < top_k ? n_c : top_k;
     if (cnt < 0 || cnt > cnt_max) {
         if (split == 0 && g == 0 && tid == 0) set_status(status, QSA_DEV_BAD_SEL);
         cnt = cnt < 0 ? 0 : cnt_max;
@@ -225,7 +227,7 @@ k_sparse_attn(const uint4* __restrict__ q, const uint16_t* __restrict__ k_cache,
         const int a = a0 + k;
         int b = n_c;  // the partial block
         if (a < cnt) {
-            b = sel_idx[(int64_t)i * kTopK + a];
+            b = sel_idx[(int64_t)i * kSelCap + a];
             if (b < 0 || b >= n_c) {
                 set_status(status, QSA_DEV_BAD_SEL);
                 b = -1;
@@ -236,18 +238,18 @@ k_sparse_attn(const uint4* __restrict__ q, const uint16_t* __restrict__ k_cache,
     __syncthreads();
 
     const int64_t kv_base = ok ? ((int64_t)s * n_kv_heads + g) * kv_capacity * kHeadDim : 0;
-    const int n_tiles = (n_blk + kTileBlocks - 1) / kTileBlocks;
+    const int n_tiles = (n_blk + ipt - 1) / ipt;
 
     auto load_tile = [&](int tile, int stage) {
 #pragma unroll
         for (int k = 0; k < (kTileTok * 16) / kThreads; ++k) {
             const int idx = tid + k * kThreads;
             const int row = idx >> 4, ch = idx & 15;
-            const int bl = tile * kTileBlocks + (row >> 2);
-            const int tin = row & 3;
+            const int bl = tile * ipt + (row >> bs_log2);
+            const int tin = row & (bs - 1);
             const int b = bl < n_blk ? s_blk[bl] : -1;
             const bool valid = b >= 0 && (a0 + bl < cnt || tin < n_part);
-            const int64_t off = valid ? kv_base + ((int64_t)b * kBlock + tin) * kHeadDim + ch * 8 : 0;
+            const int64_t off = valid ? kv_base + (((int64_t)b << bs_log2) + tin) * kHeadDim + ch * 8 : 0;
             const uint32_t so = swz(row, ch) + stage * kStageBytes;
             cp_async16(sbase + kSmemK + so, k_cache + off, valid ? 16 : 0);
             cp_async16(sbase + kSmemV + so, v_cache + off, valid ? 16 : 0);
@@ -461,21 +463,6 @@ k_sparse_attn(const uint4* __restrict__ q, const uint16_t* __restrict__ k_cache,
     else merge_splits<16>(partial + pair * n_split * pstride, n_split, G, out + ((int64_t)i * n_q_heads + g * G) * kHeadDim);
 }
 
-int attn_splits(int32_t n_q, int32_t n_kv_heads)
-{
-    // Split each (query, KV head) block list so that the whole grid is one wave at two
-    // CTAs per SM (shared memory allows two) on the 148 SMs of a B200: long CTAs keep
-    // three K/V stages in flight instead of paying their set-up and merge per tile.
-    constexpr int64_t kSlots = 2 * 148;
-    const int64_t tiles_max = (kMaxSplitBlocks + kTileBlocks - 1) / kTileBlocks;  // 33
-    const int64_t pairs = (int64_t)n_q * n_kv_heads;
-    int64_t want = pairs > 0 ? kSlots / pairs : 1;
-    if (want < 1) want = 1;
-    if (want > kMaxClusterSplits) want = kMaxClusterSplits;  // the splits of a pair form one cluster
-    const int64_t tiles_per = (tiles_max + want - 1) / want;
-    return (int)((tiles_max + tiles_per - 1) / tiles_per);
-}
-
 cudaError_t launch_attention(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,
                              const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,
                              const int32_t* sel_cnt, int32_t n_q, void* out, int n_split, float* partial,
@@ -483,8 +470,11 @@ cudaError_t launch_attention(const qsa_dims& d, const void* q, const void* k_cac
 {
     if (n_q <= 0) return cudaSuccess;
     if (n_split > kMaxClusterSplits) return cudaErrorInvalidValue;
+    int bs_log2 = 0;
+    while ((1 << bs_log2) < d.block_size) ++bs_log2;
+    const int ipt = kTileTok >> bs_log2;
     const int bps = (kMaxSplitBlocks + n_split - 1) / n_split;
-    const int bps_tiles = ((bps + kTileBlocks - 1) / kTileBlocks) * kTileBlocks;
+    const int bps_tiles = ((bps + ipt - 1) / ipt) * ipt;
     const float scale = d.softmax_scale > 0.f ? d.softmax_scale : 1.0f / sqrtf((float)d.head_dim);
     const float scale_log2 = scale * 1.4426950408889634f;
     static std::atomic<bool> attr_set[128];  // per device; setting it twice is harmless
@@ -520,7 +510,8 @@ cudaError_t launch_attention(const qsa_dims& d, const void* q, const void* k_cac
     cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, k_sparse_attn, (const uint4*)q, (const uint16_t*)k_cache,
                               (const uint16_t*)v_cache, q_seq, q_pos, sel_idx, sel_cnt, d.batch, d.n_q_heads,
-                              d.n_kv_heads, d.kv_capacity, scale_log2, bps_tiles, n_split, clustered ? 1 : 0,
+                              d.n_kv_heads, d.kv_capacity, bs_log2, d.top_k, scale_log2, bps_tiles, n_split,
+                              clustered ? 1 : 0,
                               (__nv_bfloat16*)out, partial, counters, status);
 }
 

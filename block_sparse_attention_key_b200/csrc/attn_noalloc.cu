@@ -84,11 +84,10 @@ extern "C" int qsa_sparse_attn_noalloc(const qsa_dims* dims, const void* q, cons
         !aligned16(sel_idx) || !aligned16(sel_cnt) || !aligned16(out))
         return QSA_ERR_INVALID_ARG;
 
-    const int n_split = attn_splits(n_q, dims->n_kv_heads);
-    const size_t counter_bytes = ((size_t)n_q * dims->n_kv_heads * 4 + kCounterAlign - 1) / kCounterAlign *
-                                 kCounterAlign;
-    const size_t partial_bytes =
-        n_split > 1 ? (size_t)n_q * dims->n_kv_heads * n_split * (32 + 16 * kHeadDim) * 4 : 0;
+    const int64_t pairs = (int64_t)n_q * dims->n_kv_heads;
+    const int n_split = attn_decode_split_bound(pairs);
+    const size_t counter_bytes = ((size_t)pairs * 4 + kCounterAlign - 1) / kCounterAlign * kCounterAlign;
+    const size_t partial_bytes = n_split > 1 ? attn_decode_partial_bytes() : 0;
     if (counter_bytes + partial_bytes > kScratchBytes) return QSA_ERR_WORKSPACE_TOO_SMALL;
 
     cudaStream_t st = (cudaStream_t)stream;
@@ -96,10 +95,10 @@ extern "C" int qsa_sparse_attn_noalloc(const qsa_dims* dims, const void* q, cons
     if (scratch_address(st, &base) != cudaSuccess) return QSA_ERR_CUDA;
     unsigned* counters = (unsigned*)base;
     float* partial = (float*)((char*)base + counter_bytes);
-    if (n_split > 1 && cudaMemsetAsync(counters, 0, (size_t)n_q * dims->n_kv_heads * 4, st) != cudaSuccess)
-        return QSA_ERR_CUDA;
-    // no status word in this variant: out-of-range indices are still skipped, just not reported
-    const cudaError_t e = launch_attention(*dims, q, k_cache, v_cache, q_seq, q_pos, sel_idx, sel_cnt, n_q, out,
-                                           n_split, partial, counters, nullptr, st, false, false);
+    if (n_split > 1 && cudaMemsetAsync(counters, 0, (size_t)pairs * 4, st) != cudaSuccess) return QSA_ERR_CUDA;
+    // no status word in this variant: out-of-range indices are still skipped, just not
+    // reported; split partials always meet through the scratch array
+    const cudaError_t e = launch_attn_decode(*dims, q, k_cache, v_cache, q_seq, q_pos, sel_idx, sel_cnt, nullptr, 0,
+                                             0, n_q, 1, out, partial, counters, nullptr, st, false, false, true);
     return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
 }

@@ -6,8 +6,8 @@
 // The pooled cache holds one bf16 mean key per complete block and is extended
 // as tokens are appended, so each block is pooled exactly once.
 //
-// HBM-bound and tiny (<= 2,048 blocks x 640 B per call): one thread per
-// (block, 8-dim chunk), four 16-byte loads and one 16-byte store.  The same
+// HBM-bound and tiny: one thread per (block, 8-dim chunk), one 16-byte load per
+// token of the block (4 in the published setting) and one 16-byte store.  The same
 // launch clears the layer call's select control blocks and split counters, so
 // the decode chain needs no separate memset.
 
@@ -18,7 +18,7 @@ namespace qsa {
 __global__ void __launch_bounds__(256)
 k_pool_append(const uint4* __restrict__ idx_k, uint4* __restrict__ pooled,
               const int32_t* __restrict__ len_before, const int32_t* __restrict__ len_after,
-              int64_t kv_capacity, int32_t max_new_tokens, int32_t max_new_blocks, int pool_ctas,
+              int64_t kv_capacity, int bs, int32_t max_new_tokens, int32_t max_new_blocks, int pool_ctas,
               uint4* __restrict__ zero, int64_t zero_words, unsigned* status)
 {
     griddep_wait();
@@ -35,7 +35,7 @@ k_pool_append(const uint4* __restrict__ idx_k, uint4* __restrict__ pooled,
         if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, QSA_DEV_BAD_LEN);
         return;
     }
-    int n = la / kBlock - lb / kBlock;
+    int n = la / bs - lb / bs;
     if (la - lb > max_new_tokens) {
         if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, QSA_DEV_TOO_MANY_NEW);
         n = min(n, max_new_blocks);
@@ -44,15 +44,15 @@ k_pool_append(const uint4* __restrict__ idx_k, uint4* __restrict__ pooled,
     const int j = gid >> 3;          // which appended block
     const int c = gid & 7;           // which 8-dim chunk of the 64-dim key
     if (j >= n) return;
-    const int64_t b = (int64_t)(lb / kBlock) + j;
-    const int64_t nb_cap = kv_capacity / kBlock;
+    const int64_t b = (int64_t)(lb / bs) + j;
+    const int64_t nb_cap = kv_capacity / bs;
     // 8 uint4 chunks per 64-dim bf16 row
-    const uint4* src = idx_k + ((int64_t)s * kv_capacity + b * kBlock) * 8 + c;
+    const uint4* src = idx_k + ((int64_t)s * kv_capacity + b * bs) * 8 + c;
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll
-    for (int tok = 0; tok < kBlock; ++tok) {
+#pragma unroll 4
+    for (int tok = 0; tok < bs; ++tok) {
         const uint4 v = __ldg(src + tok * 8);
         const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -61,11 +61,13 @@ k_pool_append(const uint4* __restrict__ idx_k, uint4* __restrict__ pooled,
             acc[2 * e + 1] += bf16hi(w4[e]);
         }
     }
+    // the block size is a power of two: the reciprocal is exact and the mean rounds once
+    const float inv = 1.0f / (float)bs;
     uint32_t o[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-        const __nv_bfloat16 lo = __float2bfloat16_rn(acc[2 * e] * 0.25f);
-        const __nv_bfloat16 hi = __float2bfloat16_rn(acc[2 * e + 1] * 0.25f);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(acc[2 * e] * inv);
+        const __nv_bfloat16 hi = __float2bfloat16_rn(acc[2 * e + 1] * inv);
         o[e] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
     }
     pooled[((int64_t)s * nb_cap + b) * 8 + c] = make_uint4(o[0], o[1], o[2], o[3]);
@@ -75,14 +77,14 @@ cudaError_t launch_pool(const qsa_dims& d, const void* idx_k, void* pooled, cons
                         const int32_t* len_after, int32_t max_new_tokens, void* zero, size_t zero_bytes,
                         unsigned* status, cudaStream_t st)
 {
-    const int32_t max_new_blocks = max_new_tokens > 0 ? max_new_tokens / kBlock + 1 : 0;
+    const int32_t max_new_blocks = max_new_tokens > 0 ? max_new_tokens / d.block_size + 1 : 0;
     const int pool_ctas = (int)(((int64_t)max_new_blocks * 8 + 255) / 256);
     const int64_t zero_words = zero ? (int64_t)(zero_bytes / 16) : 0;
     const int zero_ctas = (int)((zero_words + 1023) / 1024);  // 4 stores per thread
     const int ctas = pool_ctas > zero_ctas ? pool_ctas : zero_ctas;
     if (ctas == 0) return cudaSuccess;
     return launch_k(k_pool_append, dim3((unsigned)ctas, (unsigned)d.batch), dim3(256), 0, st, false,
-                    (const uint4*)idx_k, (uint4*)pooled, len_before, len_after, d.kv_capacity, max_new_tokens,
+                    (const uint4*)idx_k, (uint4*)pooled, len_before, len_after, d.kv_capacity, d.block_size, max_new_tokens,
                     max_new_blocks, pool_ctas, (uint4*)zero, zero_words, status);
 }
 

@@ -1,5 +1,5 @@
 // Prefill indexer scoring and top-512 selection on the tcgen05 tensor cores
-// (steps 2 and 3 of the QSA layer for a chunk of queries of one sequence).
+// (steps 2 and 3 of the QSA layer for chunks of queries: prefill).
 //
 // blog.cecily.jp/6295 (Raschka's explainer paragraph) and keieiax.jp glossary
 // "Qwen Sparse Attention" (section on 4-token micro-blocks): every query scores
@@ -9,6 +9,10 @@
 // score = sum_h w_h ReLU(S_h).  The score matrix (8 GiB at 8,192 queries x 1M
 // tokens) is never stored: each CTA streams its range of pooled keys and keeps,
 // per query row, only the blocks that can still be in the row's top 512.
+//
+// A 128-query tile may hold rows of several sequences (ragged chunks in one call):
+// the CTA then makes one pass over the pooled keys per distinct sequence, and a row
+// scores only in its own sequence's pass.
 //
 // CTA = 10 warps, one CTA per SM (512 TMEM columns):
 //   warp 0      TMA producer: the 4 query tiles once, then 64-block pooled tiles
@@ -73,12 +77,15 @@ struct __align__(1024) K3Smem {
     uint32_t hist[2][kHistBins][kM];            // 64 KiB, counter-major per warpgroup
     float w[kM][kIdxHeads];
     int n_c[kM];
+    int row_seq[kM];     // sequence of each row, -1 for rows that score nothing
+    int pass_seq[kM];    // distinct sequences of the tile, in order of first appearance
+    int pass_ncmax[kM];  // longest row of each pass
+    int n_pass;
     uint64_t full[kNumB], empty[kNumB];
     uint64_t tmem_full[2], tmem_empty[2];
     uint64_t a_full, mma_done;
     uint32_t tmem_base;
     int error;
-    int nc_max, seq;
 };
 
 __device__ __forceinline__ uint64_t now_ns()
@@ -173,7 +180,7 @@ __global__ void __launch_bounds__(kK3Threads, 1)
 k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_p,
                     const float* __restrict__ w, const int32_t* __restrict__ q_seq,
                     const int32_t* __restrict__ q_pos, int32_t n_q, int32_t batch, int64_t kv_capacity,
-                    int64_t max_blocks, int n_split, int seg_cap, uint32_t* __restrict__ shist,
+                    int64_t max_blocks, int bs, int top_k, int n_split, int seg_cap, uint32_t* __restrict__ shist,
                     unsigned long long* __restrict__ cand, unsigned* __restrict__ cand_cnt,
                     unsigned* __restrict__ theta_g, unsigned* status)
 {
@@ -197,32 +204,52 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
         mbar_init(&S.a_full, 1);
         mbar_init(&S.mma_done, 1);
         S.error = 0;
-        S.nc_max = 0;
-        S.seq = q_seq[row0];
         fence_mbar_init();
     }
     for (int k = tid; k < 2 * kHistBins * kM; k += kK3Threads) (&S.hist[0][0][0])[k] = 0;
-    __syncthreads();
     if (tid < kM) {
         const int64_t r = row0 + tid;
-        int nc = 0;
+        int nc = 0, seq = -1;
         if (r < n_q) {
             const int s = q_seq[r], t = q_pos[r];
-            const bool ok = s == S.seq && s >= 0 && s < batch && t >= 0 && (int64_t)t < kv_capacity;
-            if (!ok && split == 0 && !kSample) set_status(status, s != S.seq ? QSA_DEV_BAD_SEQ : QSA_DEV_BAD_POS);
+            const bool ok = s >= 0 && s < batch && t >= 0 && (int64_t)t < kv_capacity;
+            if (!ok && split == 0 && !kSample) set_status(status, (s < 0 || s >= batch) ? QSA_DEV_BAD_SEQ : QSA_DEV_BAD_POS);
             if (ok) {
-                int64_t c = ((int64_t)t + 1) / kBlock;
+                int64_t c = ((int64_t)t + 1) / bs;
                 if (c > max_blocks) {
                     if (split == 0 && !kSample) set_status(status, QSA_DEV_BLOCKS_OVER);
                     c = max_blocks;
                 }
                 nc = (int)c;
+                seq = nc > 0 ? s : -1;
             }
 #pragma unroll
             for (int h = 0; h < kIdxHeads; ++h) S.w[tid][h] = w[r * kIdxHeads + h];
         }
         S.n_c[tid] = nc;
-        if (r < n_q) atomicMax(&S.nc_max, nc);
+        S.row_seq[tid] = seq;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        // one pass over the pooled keys per distinct sequence of the tile (a chunk of one
+        // sequence: a single pass; a tile straddling two chunks: two)
+        int np = 0;
+        for (int r = 0; r < kM; ++r) {
+            const int sq = S.row_seq[r];
+            if (sq < 0) continue;
+            int p = np - 1;
+            if (p < 0 || S.pass_seq[p] != sq) {
+                p = 0;
+                while (p < np && S.pass_seq[p] != sq) ++p;
+                if (p == np) {
+                    S.pass_seq[np] = sq;
+                    S.pass_ncmax[np] = 0;
+                    ++np;
+                }
+            }
+            S.pass_ncmax[p] = max(S.pass_ncmax[p], S.n_c[r]);
+        }
+        S.n_pass = np;
     }
     if (warp == 1) {
         tmem_alloc(&S.tmem_base, kTmemCols);
@@ -232,16 +259,26 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
     __syncthreads();
     tc_fence_after();
 
-    // this CTA's range of scored positions (every bstride-th block when sampling):
-    // a 1/n_split share of the tile's longest row
-    const int nc_max = (S.nc_max + bstride - 1) / bstride;
-    const int chunk = (((nc_max + n_split - 1) / n_split) + kN - 1) / kN * kN;
-    const int blk0 = split * chunk;
-    const int blk1 = min(blk0 + chunk, nc_max);
-    const int n_stages = blk1 > blk0 ? (blk1 - blk0 + kN - 1) / kN : 0;
+    // per pass, this CTA's range of scored positions (every bstride-th block when
+    // sampling): a 1/n_split share of the pass's longest row; stages are numbered
+    // across passes (J) for the ring slots and the TMEM stages
+    const int n_pass = S.n_pass;
+    auto pass_range = [&](int p, int& blk0, int& n_st) {
+        const int ncm = (S.pass_ncmax[p] + bstride - 1) / bstride;
+        const int chunk = (((ncm + n_split - 1) / n_split) + kN - 1) / kN * kN;
+        blk0 = split * chunk;
+        const int blk1 = min(blk0 + chunk, ncm);
+        n_st = blk1 > blk0 ? (blk1 - blk0 + kN - 1) / kN : 0;
+    };
+    int n_stages = 0;
+    for (int p = 0; p < n_pass; ++p) {
+        int b0_, n_st;
+        pass_range(p, b0_, n_st);
+        n_stages += n_st;
+    }
     const uint32_t tmem = S.tmem_base;
     volatile int* err = &S.error;
-    const int64_t prow0 = (int64_t)S.seq * (kv_capacity / kBlock) / bstride;
+    const int64_t seq_rows = (kv_capacity / bs) / bstride;  // pooled rows per sequence in the view
 
     if (warp == 0) {
         if (lane == 0 && n_stages > 0) {
@@ -250,12 +287,17 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
             mbar_arrive_expect_tx(&S.a_full, kIdxHeads * kM * kIdxDim * 2);
             for (int h = 0; h < kIdxHeads; ++h) tma_load_3d(S.a[h], &tmap_q, &S.a_full, 0, h, (int)row0);
             int issued = 0;
-            for (int j = 0; j < n_stages; ++j) {
-                const int slot = j % kNumB;
-                if (j >= kNumB && !wait_phase(&S.empty[slot], ((j / kNumB) - 1) & 1, err, status)) break;
-                mbar_arrive_expect_tx(&S.full[slot], kN * kIdxDim * 2);
-                tma_load_2d(S.b[slot], &tmap_p, &S.full[slot], 0, (int)(prow0 + blk0 + (int64_t)j * kN));
-                issued = j + 1;
+            for (int p = 0, J = 0; p < n_pass && !*err; ++p) {
+                int blk0, n_st;
+                pass_range(p, blk0, n_st);
+                const int64_t prow0 = (int64_t)S.pass_seq[p] * seq_rows;
+                for (int j = 0; j < n_st; ++j, ++J) {
+                    const int slot = J % kNumB;
+                    if (J >= kNumB && !wait_phase(&S.empty[slot], ((J / kNumB) - 1) & 1, err, status)) break;
+                    mbar_arrive_expect_tx(&S.full[slot], kN * kIdxDim * 2);
+                    tma_load_2d(S.b[slot], &tmap_p, &S.full[slot], 0, (int)(prow0 + blk0 + (int64_t)j * kN));
+                    issued = J + 1;
+                }
             }
             if (*err) {
                 // drain: every issued tile and the query tiles must land before the CTA exits
@@ -276,7 +318,7 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
 #pragma unroll
             for (int h = 0; h < kIdxHeads; ++h) adesc[h] = smem_desc_sw128(smem_u32(S.a[h]));
             if (wait_phase(&S.a_full, 0, err, status)) {
-                for (int j = 0; j < n_stages; ++j) {
+                for (int j = 0; j < n_stages; ++j) {  // every pass's stages in order
                     const int slot = j % kNumB, ts = j & 1;
                     if (!wait_phase(&S.full[slot], (j / kNumB) & 1, err, status)) break;
                     if (j >= 2 && !wait_phase(&S.tmem_empty[ts], ((j >> 1) - 1) & 1, err, status)) break;
@@ -305,8 +347,9 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const int64_t row_g = row0 + row;
-        const int nc = (S.n_c[row] + bstride - 1) / bstride;  // scored positions of this row
-        const bool live = row_g < n_q && nc > 0;
+        const int nc_own = (S.n_c[row] + bstride - 1) / bstride;  // scored positions of this row
+        const int my_seq = S.row_seq[row];
+        const bool live_any = row_g < n_q && nc_own > 0;
         const float wf0 = S.w[row][0], wf1 = S.w[row][1], wf2 = S.w[row][2], wf3 = S.w[row][3];
         const unsigned long long w0 = pack2(wf0, wf0), w1 = pack2(wf1, wf1), w2 = pack2(wf2, wf2),
                                  w3 = pack2(wf3, wf3);
@@ -319,7 +362,7 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
         unsigned long long* seg = cand + ((row_g * n_split + split) * 2 + wg) * (int64_t)seg_cap;
         unsigned theta_key = 0x00800000u;  // key of -FLT_MAX: every finite score passes
         unsigned cnt = 0, since = 0;
-        if (!kSample && shist && live && S.n_c[row] > 2 * kTopK) {
+        if (!kSample && shist && live_any && S.n_c[row] > 2 * top_k) {
             // starting threshold: lower edge of the bin holding the row's kSampleKth-best
             // sampled score (merge of the windows of every sampling CTA and warpgroup;
             // a window that saw no sample has base kNoWindow)
@@ -348,127 +391,140 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
         }
         float theta_f = key_to_float(theta_key);
 
-        for (int j = wg; j < n_stages; j += 2) {
-            const int k_own = j >> 1;  // this warpgroup's k-th tile
-            if (!wait_phase(&S.tmem_full[wg], k_own & 1, err, status)) break;
-            tc_fence_after();
-            if (!kSample && (k_own & 7) == 7 && live) {
-                const unsigned g = __ldcg(theta_g + row_g);
-                if (g > theta_key) {
-                    theta_key = g;
-                    theta_f = key_to_float(theta_key);
+        bool stop = false;
+        for (int p = 0, J = 0; p < n_pass && !stop; ++p) {
+            int blk0, n_st;
+            pass_range(p, blk0, n_st);
+            // rows of other sequences score nothing in this pass
+            const int nc = my_seq == S.pass_seq[p] ? nc_own : 0;
+            const bool live = live_any && nc > 0;
+            for (int jp = 0; jp < n_st; ++jp, ++J) {
+                if ((J & 1) != wg) continue;
+                const int j = jp;          // stage within the pass
+                const int k_own = J >> 1;  // this warpgroup's k-th tile
+                if (!wait_phase(&S.tmem_full[wg], k_own & 1, err, status)) {
+                    stop = true;
+                    break;
                 }
-            }
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                float a[kIdxHeads][32];
-#pragma unroll
-                for (int h = 0; h < kIdxHeads; ++h) {
-                    float lo[16], hi[16];
-                    tmem_ld16(tbase + h * kN + half * 32, lo);
-                    tmem_ld16(tbase + h * kN + half * 32 + 16, hi);
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        a[h][c] = lo[c];
-                        a[h][16 + c] = hi[c];
+                tc_fence_after();
+                if (!kSample && (k_own & 7) == 7 && live) {
+                    const unsigned g = __ldcg(theta_g + row_g);
+                    if (g > theta_key) {
+                        theta_key = g;
+                        theta_f = key_to_float(theta_key);
                     }
                 }
-                tmem_ld_wait();
-                if (half == 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&S.tmem_empty[wg]);
-                }
-                if (!live) continue;
-                float sc[32];
-                row_scores32(a, w0, w1, w2, w3, sc);
-                const int b_base = blk0 + j * kN + half * 32;
-                if (b_base + 32 > nc) {
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float a[kIdxHeads][32];
 #pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        if (b_base + c >= nc) sc[c] = -INFINITY;
-                }
-                if (kSample) {
-                    // histogram of every sampled score within 4 octaves of the largest seen
+                    for (int h = 0; h < kIdxHeads; ++h) {
+                        float lo[16], hi[16];
+                        tmem_ld16(tbase + h * kN + half * 32, lo);
+                        tmem_ld16(tbase + h * kN + half * 32 + 16, hi);
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) {
+                            a[h][c] = lo[c];
+                            a[h][16 + c] = hi[c];
+                        }
+                    }
+                    tmem_ld_wait();
+                    if (half == 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&S.tmem_empty[wg]);
+                    }
+                    if (!live) continue;
+                    float sc[32];
+                    row_scores32(a, w0, w1, w2, w3, sc);
+                    const int b_base = blk0 + j * kN + half * 32;
+                    if (b_base + 32 > nc) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            if (b_base + c >= nc) sc[c] = -INFINITY;
+                    }
+                    if (kSample) {
+                        // histogram of every sampled score within 4 octaves of the largest seen
+                        float m = sc[0];
+#pragma unroll
+                        for (int c = 1; c < 31; c += 2) m = max3(m, sc[c], sc[c + 1]);
+                        m = fmaxf(m, sc[31]);
+                        if (m == -INFINITY) continue;
+                        if (wb < 0) wb = max((int)(orderable_key(m) >> kSampleShift) - (kHistBins - 4), 0);
+                        const int top = (int)(orderable_key(m) >> kSampleShift);
+                        if (top - wb >= kHistBins) {  // slide the window up under the largest score
+                            const int d = top - wb - (kHistBins - 4);
+                            for (int k = 0; k < kHistBins; ++k) hist[k * kM] = k + d < kHistBins ? hist[(k + d) * kM] : 0u;
+                            wb += d;
+                        }
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            const int jj = (int)(orderable_key(sc[c]) >> kSampleShift) - wb;
+                            if (sc[c] != -INFINITY && jj >= 0) hist[jj * kM] += 1;
+                        }
+                        continue;
+                    }
                     float m = sc[0];
 #pragma unroll
                     for (int c = 1; c < 31; c += 2) m = max3(m, sc[c], sc[c + 1]);
                     m = fmaxf(m, sc[31]);
-                    if (m == -INFINITY) continue;
-                    if (wb < 0) wb = max((int)(orderable_key(m) >> kSampleShift) - (kHistBins - 4), 0);
-                    const int top = (int)(orderable_key(m) >> kSampleShift);
-                    if (top - wb >= kHistBins) {  // slide the window up under the largest score
-                        const int d = top - wb - (kHistBins - 4);
-                        for (int k = 0; k < kHistBins; ++k) hist[k * kM] = k + d < kHistBins ? hist[(k + d) * kM] : 0u;
-                        wb += d;
-                    }
+                    if (!(m >= theta_f)) continue;
+                    unsigned pass = 0;
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const int jj = (int)(orderable_key(sc[c]) >> kSampleShift) - wb;
-                        if (sc[c] != -INFINITY && jj >= 0) hist[jj * kM] += 1;
-                    }
-                    continue;
-                }
-                float m = sc[0];
-#pragma unroll
-                for (int c = 1; c < 31; c += 2) m = max3(m, sc[c], sc[c + 1]);
-                m = fmaxf(m, sc[31]);
-                if (!(m >= theta_f)) continue;
-                unsigned pass = 0;
-#pragma unroll
-                for (int c = 0; c < 32; ++c) pass |= (sc[c] >= theta_f ? 1u : 0u) << c;
-                // admissions: columns in increasing block order
-                while (pass) {
-                    const int c = __ffs(pass) - 1;
-                    pass &= pass - 1;
-                    const float sv = pick32(sc, c);
-                    if (!(sv >= theta_f)) continue;  // the threshold may have risen within this tile
-                    const unsigned key = orderable_key(sv);
-                    if (cnt < (unsigned)seg_cap) seg[cnt] = ((unsigned long long)key << 32) | (unsigned)(b_base + c);
-                    ++cnt;
-                    // the raise histogram only matters once this segment holds many blocks
-                    if (cnt < (unsigned)(kTopK >> 1)) continue;
-                    const int bin = (int)(key >> kHistShift);
-                    if (wb < 0) wb = max(bin - 56, 0);
-                    int jj = bin - wb;
-                    if (jj >= kHistBins) {  // keep the window under the largest score seen
-                        const int d = jj - 56;
-                        unsigned kept = 0;
-                        for (int k = 0; k < kHistBins; ++k) {
-                            const unsigned v = k + d < kHistBins ? hist[(k + d) * kM] : 0u;
-                            hist[k * kM] = v;
-                            kept += v;
-                        }
-                        wcount = kept;
-                        wb += d;
-                        jj = 56;
-                    }
-                    if (jj >= 0) {
-                        hist[jj * kM] += 1;
-                        ++wcount;
-                    }
-                    if (++since >= kRaiseEvery && wcount >= (unsigned)kTopK + kRaiseEvery) {
-                        since = 0;
-                        // largest q with (keys counted in bins >= q) >= top_k, scanning up from the bottom
-                        unsigned above = wcount;
-                        int q = 0;
-                        while (q < kHistBins - 1) {
-                            const unsigned hq = hist[q * kM];
-                            if (above - hq < (unsigned)kTopK) break;
-                            above -= hq;
-                            ++q;
-                        }
-                        if (q >= 1) {
-                            const unsigned edge_key = (unsigned)(wb + q) << kHistShift;
-                            if (edge_key + 1 > theta_key) {
-                                theta_key = edge_key + 1;  // strict for this thread's later blocks
-                                theta_f = key_to_float(theta_key);
+                    for (int c = 0; c < 32; ++c) pass |= (sc[c] >= theta_f ? 1u : 0u) << c;
+                    // admissions: columns in increasing block order
+                    while (pass) {
+                        const int c = __ffs(pass) - 1;
+                        pass &= pass - 1;
+                        const float sv = pick32(sc, c);
+                        if (!(sv >= theta_f)) continue;  // the threshold may have risen within this tile
+                        const unsigned key = orderable_key(sv);
+                        if (cnt < (unsigned)seg_cap) seg[cnt] = ((unsigned long long)key << 32) | (unsigned)(b_base + c);
+                        ++cnt;
+                        // the raise histogram only matters once this segment holds many blocks
+                        if (cnt < (unsigned)(top_k >> 1)) continue;
+                        const int bin = (int)(key >> kHistShift);
+                        if (wb < 0) wb = max(bin - 56, 0);
+                        int jj = bin - wb;
+                        if (jj >= kHistBins) {  // keep the window under the largest score seen
+                            const int d = jj - 56;
+                            unsigned kept = 0;
+                            for (int k = 0; k < kHistBins; ++k) {
+                                const unsigned v = k + d < kHistBins ? hist[(k + d) * kM] : 0u;
+                                hist[k * kM] = v;
+                                kept += v;
                             }
-                            atomicMax(theta_g + row_g, edge_key);
-                            for (int k = 0; k < kHistBins; ++k)
-                                hist[k * kM] = k + q < kHistBins ? hist[(k + q) * kM] : 0u;
-                            wcount = above;
-                            wb += q;
+                            wcount = kept;
+                            wb += d;
+                            jj = 56;
+                        }
+                        if (jj >= 0) {
+                            hist[jj * kM] += 1;
+                            ++wcount;
+                        }
+                        if (++since >= kRaiseEvery && wcount >= (unsigned)top_k + kRaiseEvery) {
+                            since = 0;
+                            // largest q with (keys counted in bins >= q) >= top_k, scanning up from the bottom
+                            unsigned above = wcount;
+                            int q = 0;
+                            while (q < kHistBins - 1) {
+                                const unsigned hq = hist[q * kM];
+                                if (above - hq < (unsigned)top_k) break;
+                                above -= hq;
+                                ++q;
+                            }
+                            if (q >= 1) {
+                                const unsigned edge_key = (unsigned)(wb + q) << kHistShift;
+                                if (edge_key + 1 > theta_key) {
+                                    theta_key = edge_key + 1;  // strict for this thread's later blocks
+                                    theta_f = key_to_float(theta_key);
+                                }
+                                atomicMax(theta_g + row_g, edge_key);
+                                for (int k = 0; k < kHistBins; ++k)
+                                    hist[k * kM] = k + q < kHistBins ? hist[(k + q) * kM] : 0u;
+                                wcount = above;
+                                wb += q;
+                            }
                         }
                     }
                 }
@@ -551,7 +607,7 @@ __device__ __forceinline__ void gather_segments(const unsigned long long* __rest
 // go to the worklist of k_prefill_fallback.
 __global__ void __launch_bounds__(256)
 k_prefill_finish(const int32_t* __restrict__ q_seq, const int32_t* __restrict__ q_pos, int32_t n_q, int32_t batch,
-                 int64_t kv_capacity, int64_t max_blocks, int n_split, int seg_cap,
+                 int64_t kv_capacity, int64_t max_blocks, int bs, int top_k, int n_split, int seg_cap,
                  const unsigned long long* __restrict__ cand, const unsigned* __restrict__ cand_cnt,
                  const unsigned* __restrict__ theta_g, int32_t* __restrict__ worklist, int32_t* __restrict__ sel_idx,
                  int32_t* __restrict__ sel_cnt)
@@ -561,13 +617,12 @@ k_prefill_finish(const int32_t* __restrict__ q_seq, const int32_t* __restrict__ 
     __shared__ int s_n, s_fail;
     const int tid = threadIdx.x;
     const int64_t r = blockIdx.x;
-    const int tile_seq = q_seq[(r / kM) * kM];
     const int s = q_seq[r], t = q_pos[r];
-    const bool ok = s == tile_seq && s >= 0 && s < batch && t >= 0 && (int64_t)t < kv_capacity;
-    const int64_t n_c = ok ? min(((int64_t)t + 1) / kBlock, max_blocks) : 0;
-    int32_t* out = sel_idx + r * kTopK;
-    if (n_c <= kTopK) {
-        for (int k = tid; k < kTopK; k += 256) out[k] = k < n_c ? k : -1;
+    const bool ok = s >= 0 && s < batch && t >= 0 && (int64_t)t < kv_capacity;
+    const int64_t n_c = ok ? min(((int64_t)t + 1) / bs, max_blocks) : 0;
+    int32_t* out = sel_idx + r * kSelCap;
+    if (n_c <= top_k) {
+        for (int k = tid; k < kSelCap; k += 256) out[k] = k < n_c ? k : -1;
         if (tid == 0) sel_cnt[r] = (int)n_c;
         return;
     }
@@ -576,12 +631,12 @@ k_prefill_finish(const int32_t* __restrict__ q_seq, const int32_t* __restrict__ 
         s_n = 0;
         s_fail = 0;
     }
-    for (int k = tid; k < kTopK; k += 256) S.list[k] = INT_MAX;
+    for (int k = tid; k < kSelCap; k += 256) S.list[k] = INT_MAX;
     if (tid == 0) S.n_list = 0;
     __syncthreads();
     gather_segments(cand, cand_cnt, r, n_split, seg_cap, theta, s_cand, &s_n, &s_fail);
     const int nc = s_n;
-    if (s_fail || nc > kCandCap || nc < kTopK) {
+    if (s_fail || nc > kCandCap || nc < top_k) {
         if (tid == 0) worklist[1 + atomicAdd(worklist, 1)] = (int32_t)r;
         return;
     }
@@ -591,14 +646,14 @@ k_prefill_finish(const int32_t* __restrict__ q_seq, const int32_t* __restrict__ 
         const int j = tid + 256 * k;
         cr[k] = j < nc ? s_cand[j] : 0ull;
     }
-    const Cut cut = resolve_cut_regs(S, cr, nc, kTopK, true, 0u);
+    const Cut cut = resolve_cut_regs(S, cr, nc, top_k, true, 0u);
     if (!take_by_cut(S, cr, nc, cut)) {
         if (tid == 0) worklist[1 + atomicAdd(worklist, 1)] = (int32_t)r;
         return;
     }
     sort_list_512(S);
-    for (int k = tid; k < kTopK; k += 256) out[k] = S.list[k];
-    if (tid == 0) sel_cnt[r] = kTopK;
+    for (int k = tid; k < kSelCap; k += 256) out[k] = k < top_k ? S.list[k] : -1;
+    if (tid == 0) sel_cnt[r] = top_k;
 }
 
 // Rows the streaming pass could not settle: recompute the row's scores with CUDA
@@ -606,7 +661,7 @@ k_prefill_finish(const int32_t* __restrict__ q_seq, const int32_t* __restrict__ 
 __global__ void __launch_bounds__(256)
 k_prefill_fallback(const __nv_bfloat16* __restrict__ q_idx, const float* __restrict__ w,
                    const __nv_bfloat16* __restrict__ pooled, const int32_t* __restrict__ q_seq,
-                   const int32_t* __restrict__ q_pos, int64_t kv_capacity, int64_t max_blocks,
+                   const int32_t* __restrict__ q_pos, int64_t kv_capacity, int64_t max_blocks, int bs, int top_k,
                    const int32_t* __restrict__ worklist, float* __restrict__ scratch, int32_t* __restrict__ sel_idx,
                    int32_t* __restrict__ sel_cnt)
 {
@@ -618,7 +673,7 @@ k_prefill_fallback(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
     for (int wi = blockIdx.x; wi < n_work; wi += gridDim.x) {
         const int64_t r = worklist[1 + wi];
         const int s = q_seq[r], t = q_pos[r];
-        const int64_t n_c = min(((int64_t)t + 1) / kBlock, max_blocks);
+        const int64_t n_c = min(((int64_t)t + 1) / bs, max_blocks);
         __syncthreads();
         for (int k = tid; k < kIdxHeads * kIdxDim; k += 256)
             s_q[k / kIdxDim][k % kIdxDim] = __bfloat162float(q_idx[r * kIdxHeads * kIdxDim + k]);
@@ -626,7 +681,7 @@ k_prefill_fallback(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
         float wv[kIdxHeads];
 #pragma unroll
         for (int h = 0; h < kIdxHeads; ++h) wv[h] = w[r * kIdxHeads + h];
-        const __nv_bfloat16* prow = pooled + (int64_t)s * (kv_capacity / kBlock) * kIdxDim;
+        const __nv_bfloat16* prow = pooled + (int64_t)s * (kv_capacity / bs) * kIdxDim;
         for (int64_t b = tid; b < n_c; b += 256) {
             float acc[kIdxHeads] = {0.f, 0.f, 0.f, 0.f};
             const uint4* pk = reinterpret_cast<const uint4*>(prow + b * kIdxDim);
@@ -649,12 +704,12 @@ k_prefill_fallback(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
         }
         __threadfence_block();
         __syncthreads();
-        for (int k = tid; k < kTopK; k += 256) S.list[k] = INT_MAX;
+        for (int k = tid; k < kSelCap; k += 256) S.list[k] = INT_MAX;
         __syncthreads();
-        select_by_rescan(S, row_scores, n_c, true, 0u, kTopK);
-        int32_t* out = sel_idx + r * kTopK;
-        const int cnt = (int)min((int64_t)kTopK, n_c);
-        for (int k = tid; k < kTopK; k += 256) out[k] = k < cnt ? S.list[k] : -1;
+        select_by_rescan(S, row_scores, n_c, true, 0u, top_k);
+        int32_t* out = sel_idx + r * kSelCap;
+        const int cnt = (int)min((int64_t)top_k, n_c);
+        for (int k = tid; k < kSelCap; k += 256) out[k] = k < cnt ? S.list[k] : -1;
         if (tid == 0) sel_cnt[r] = cnt;
     }
 }
@@ -709,7 +764,7 @@ size_t prefill_smem_bytes() { return sizeof(K3Smem) + 1024; }
 
 bool prefill_sampled(const qsa_dims& d, int64_t max_blocks)
 {
-    return d.kv_capacity % (kBlock * kSampleStride) == 0 && max_blocks > 2 * kTopK;
+    return d.kv_capacity % ((int64_t)d.block_size * kSampleStride) == 0 && max_blocks > 2 * d.top_k;
 }
 
 cudaError_t launch_prefill_select(const qsa_dims& d, const void* q_idx, const float* w, const void* pooled,
@@ -738,7 +793,7 @@ cudaError_t launch_prefill_select(const qsa_dims& d, const void* q_idx, const fl
         // pooled keys of all sequences: [B * T/4][64] bf16, box = 64 x 64 blocks; the sampling
         // view takes every kSampleStride-th block (row pitch kSampleStride x 128 B)
         const int stride = pass == 0 ? 1 : kSampleStride;
-        const cuuint64_t dims[2] = {(cuuint64_t)kIdxDim, (cuuint64_t)(d.batch * (d.kv_capacity / kBlock) / stride)};
+        const cuuint64_t dims[2] = {(cuuint64_t)kIdxDim, (cuuint64_t)(d.batch * (d.kv_capacity / d.block_size) / stride)};
         const cuuint64_t strides[1] = {(cuuint64_t)kIdxDim * 2 * stride};
         const cuuint32_t box[2] = {(cuuint32_t)kIdxDim, (cuuint32_t)kN};
         const cuuint32_t estr[2] = {1u, 1u};
@@ -757,17 +812,17 @@ cudaError_t launch_prefill_select(const qsa_dims& d, const void* q_idx, const fl
     const int n_tiles = (n_q + kM - 1) / kM;
     if (sampled)  // the main pass's CTA grid: each thread histograms its share of its row's samples
         k_prefill_scores_tc<true><<<dim3((unsigned)n_split, (unsigned)n_tiles), kK3Threads, smem, st>>>(
-            tq, ts, w, q_seq, q_pos, n_q, d.batch, d.kv_capacity, max_blocks, n_split, 0, shist, nullptr, nullptr,
-            nullptr, status);
+            tq, ts, w, q_seq, q_pos, n_q, d.batch, d.kv_capacity, max_blocks, d.block_size, d.top_k, n_split, 0,
+            shist, nullptr, nullptr, nullptr, status);
     k_prefill_scores_tc<false><<<dim3((unsigned)n_split, (unsigned)n_tiles), kK3Threads, smem, st>>>(
-        tq, tp, w, q_seq, q_pos, n_q, d.batch, d.kv_capacity, max_blocks, n_split, seg_cap,
+        tq, tp, w, q_seq, q_pos, n_q, d.batch, d.kv_capacity, max_blocks, d.block_size, d.top_k, n_split, seg_cap,
         sampled ? shist : nullptr, cand, cand_cnt, theta_g, status);
     k_prefill_finish<<<(unsigned)n_q, 256, kCandCap * sizeof(unsigned long long), st>>>(
-        q_seq, q_pos, n_q, d.batch, d.kv_capacity, max_blocks, n_split, seg_cap, cand, cand_cnt, theta_g, worklist,
-        sel_idx, sel_cnt);
+        q_seq, q_pos, n_q, d.batch, d.kv_capacity, max_blocks, d.block_size, d.top_k, n_split, seg_cap, cand,
+        cand_cnt, theta_g, worklist, sel_idx, sel_cnt);
     k_prefill_fallback<<<(unsigned)n_fallback_ctas, 256, 0, st>>>(
         (const __nv_bfloat16*)q_idx, w, (const __nv_bfloat16*)pooled, q_seq, q_pos, d.kv_capacity, max_blocks,
-        worklist, scratch, sel_idx, sel_cnt);
+        d.block_size, d.top_k, worklist, scratch, sel_idx, sel_cnt);
     return cudaGetLastError();
 }
 

@@ -11,8 +11,10 @@
 namespace qsa {
 
 // ---- fixed method parameters (validated on the host) ----
-constexpr int kBlock = 4;        // tokens per micro-block
-constexpr int kTopK = 512;       // blocks kept per query
+// micro-block size (dims.block_size) and blocks kept per query (dims.top_k) are
+// run-time values: block_size in {1, 2, 4, 8, 16}, 1 <= top_k <= kSelCap
+constexpr int kSelCap = 512;     // capacity of a query's selection (and row stride of sel_idx)
+constexpr int kMaxBlockSize = 16;
 constexpr int kIdxHeads = 4;     // indexer heads
 constexpr int kIdxDim = 64;      // indexer head dim
 constexpr int kHeadDim = 128;    // main attention head dim
@@ -102,7 +104,7 @@ struct WsLayout {
     int64_t score_ld = 0;
     int32_t score_rows = 0;
     size_t sel = 0;        // i32 [n_q][top_k] + i32 [n_q] when the caller passes none
-    size_t partial = 0;    // f32 split-K partials
+    size_t partial = 0;    // f32 split-K partials of the decode attention
     // prefill (tensor-core) select
     size_t pf_cand = 0;    // u64 [n_q][2 * pf_split][seg_cap] admitted (key << 32 | block)
     size_t pf_cnt = 0;     // u32 [n_q][2 * pf_split]
@@ -110,12 +112,12 @@ struct WsLayout {
     size_t pf_work = 0;    // i32 [1 + n_q] fallback worklist (count zeroed per call)
     size_t pf_shist = 0;   // u32 [n_q][2][65] sampled score histograms
     size_t pf_scratch = 0; // f32 [pf_fb_ctas][max_blocks]
+    size_t qpos_loc = 0;   // i32 [n_q] positions inside a context shard
     int pf_split = 0;
     int pf_fb_ctas = 0;
     size_t total = 0;
     int n_chunks = 0;
     int chunk = 0;
-    int n_split = 1;
 };
 
 // ---- host-side argument checks shared by every entry point (api.cu) ----
@@ -125,11 +127,13 @@ bool aligned16(const void* p);
 int check_dims(const qsa_dims* d);
 // Query count and candidate-block bound of a call.
 int check_rows(const qsa_dims* d, int32_t n_q, int64_t max_blocks);
+// Draft-query groups sharing one selection: group_q >= 1 divides n_q, rows per CTA <= 32.
+int check_groups(const qsa_dims* d, int32_t n_q, int32_t group_q);
+// Paged K/V (page_table may be NULL: dense caches).
+int check_pages(const qsa_dims* d, const int32_t* page_table, int32_t page_tokens, int64_t n_pages);
 
 // Chunk of candidate blocks one CTA of the decode scoring/select passes handles.
 int select_chunk(int64_t max_blocks, int32_t n_rows);
-// Split-K factor of the decode attention.
-int attn_splits(int32_t n_q, int32_t n_kv_heads);
 WsLayout plan_workspace(const qsa_dims& d, int32_t n_q, int64_t max_blocks, int32_t mode);
 
 // ---- launchers (return cudaGetLastError()) ----
@@ -143,18 +147,22 @@ cudaError_t launch_pool(const qsa_dims& d, const void* idx_k, void* pooled, cons
 // also builds the digit-1 histogram; then, with sel_idx != nullptr (needs
 // max_blocks <= 16,384) the last CTA of each row selects the row completely,
 // otherwise it resolves digit 1 for launch_topk.
+// Row r's query indexer inputs are q_idx[row0 + r], w[row0 + r]; its sequence and
+// position are q_seq / q_pos[(row0 + r) * pos_stride] (pos_stride > 1: one selection
+// per group of draft queries, made for the group's first query).
 cudaError_t launch_score_decode(const qsa_dims& d, const void* q_idx, const float* w, const void* pooled,
                                 const int32_t* q_seq, const int32_t* q_pos, int32_t row0, int32_t n_rows,
                                 int64_t max_blocks, float* scores, int64_t ld, int chunk, TopkCtrl* ctrl,
                                 int32_t* sel_idx, int32_t* sel_cnt, unsigned* status, cudaStream_t st,
-                                bool pdl = false);
+                                bool pdl = false, int pos_stride = 1);
 // Largest max_blocks for which launch_score_decode can finish the select itself.
 constexpr int64_t kScoreFinishMaxBlocks = 16384;
 
 // Radix select over score rows [0, n_rows) (query i = row0 + r).  If `hist_done`
 // the digit-1 histogram was built by the scoring kernel.
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, int32_t row0, int32_t n_rows,
-                        int64_t max_blocks, int64_t kv_capacity, int chunk, int n_chunks, TopkCtrl* ctrl,
+                        int64_t max_blocks, int64_t kv_capacity, int bs, int top_k, int chunk, int n_chunks,
+                        TopkCtrl* ctrl,
                         unsigned long long* cand, int32_t* tmp, int32_t* sel_idx, int32_t* sel_cnt, bool hist_done,
                         unsigned* status, cudaStream_t st, bool pdl = false);
 
@@ -169,6 +177,30 @@ cudaError_t launch_prefill_select(const qsa_dims& d, const void* q_idx, const fl
                                   int n_split, unsigned long long* cand, unsigned* cand_cnt, unsigned* theta_g,
                                   uint32_t* shist, int32_t* worklist, float* scratch, int n_fallback_ctas,
                                   int32_t* sel_idx, int32_t* sel_cnt, unsigned* status, cudaStream_t st);
+
+// Decode-shaped gathered attention (attn_decode.cu): groups of `group_q` queries
+// sharing one selection row, optional paged K/V.  Splits of a (group, KV head) merge
+// in a thread-block cluster when allow_cluster and the device can hold every
+// cluster at once, else through `partial` / `counters` (counters zeroed by the caller).
+int attn_decode_split_bound(int64_t pairs);
+size_t attn_decode_partial_bytes();  // bytes of `partial` any launch needs
+cudaError_t launch_attn_decode(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,
+                               const int32_t* sel_cnt, const int32_t* page_table, int page_tokens, int64_t n_pages,
+                               int64_t n_groups, int group_q, void* out, float* partial, unsigned* counters,
+                               unsigned* status, cudaStream_t st, bool pdl, bool allow_cluster,
+                               bool counters_zeroed, float* part_out = nullptr);
+
+// Context-parallel steps (cp.cu).
+size_t cp_partial_row_floats();
+cudaError_t launch_cp_local_pos(const int32_t* q_pos, int32_t n_q, int64_t tok_lo, int64_t cap_loc, int32_t* pos_loc,
+                                cudaStream_t st);
+cudaError_t launch_cp_keys(const float* scores, int64_t ld, const int32_t* sel, const int32_t* cnt, int32_t n_q,
+                           int64_t blk_lo, unsigned long long* keys, int32_t* key_cnt, cudaStream_t st);
+cudaError_t launch_cp_merge(const unsigned long long* keys_all, const int32_t* cnt_all, int n_ranks, int32_t n_q,
+                            int top_k, int64_t blk_lo, int64_t n_local, int32_t* sel_local, int32_t* cnt_local,
+                            int32_t* sel_global, int32_t* cnt_global, cudaStream_t st);
+cudaError_t launch_cp_combine(const float* parts, int n_ranks, int64_t rows, void* out, cudaStream_t st);
 
 cudaError_t launch_attention(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,
                              const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,

@@ -5,7 +5,8 @@
 // section on 4-token micro-blocks: the indexer estimates each block's importance.
 // The score of block b for query i is
 //     sum_h w[i][h] * ReLU( q_idx[i][h] . pooled[s][b] )        (4 heads x 64 dims)
-// over the complete causal blocks b < floor((t+1)/4).
+// over the complete causal blocks b < floor((t+1)/bs) (bs = micro-block size, 4 in
+// the published setting).
 //
 // A decode query reads every pooled key of its sequence once (128 B each): an HBM
 // stream of 2 multiply-adds per byte, too many for the CUDA cores to keep pace
@@ -72,7 +73,7 @@ k_score_decode(const uint4* __restrict__ q_idx, const float* __restrict__ w, con
                const int32_t* __restrict__ q_seq, const int32_t* __restrict__ q_pos, int32_t row0,
                int32_t batch, int64_t kv_capacity, int64_t max_blocks, float* __restrict__ scores,
                int64_t ld, int chunk, TopkCtrl* __restrict__ ctrl, int32_t* __restrict__ sel_idx,
-               int32_t* __restrict__ sel_cnt, unsigned* status)
+               int32_t* __restrict__ sel_cnt, unsigned* status, int pos_stride, int bs, int top_k)
 {
     extern __shared__ __align__(1024) uint8_t s_stage[];
     __shared__ FinishSmem S;  // S.hist: the digit-1 histogram of this CTA's scores
@@ -83,10 +84,10 @@ k_score_decode(const uint4* __restrict__ q_idx, const float* __restrict__ w, con
     const int r = blockIdx.y;
     const int i = row0 + r;
     // before griddep_wait: only the layer call's own inputs (rows, query, weights)
-    const int s = q_seq[i];
-    const int t = q_pos[i];
+    const int s = q_seq[(int64_t)i * pos_stride];
+    const int t = q_pos[(int64_t)i * pos_stride];
     const bool ok = (s >= 0 && s < batch && t >= 0 && (int64_t)t < kv_capacity);
-    int64_t n_c = ok ? ((int64_t)t + 1) / kBlock : 0;
+    int64_t n_c = ok ? ((int64_t)t + 1) / bs : 0;
     const bool over = n_c > max_blocks;
     if (over) n_c = max_blocks;
     const int64_t b0 = (int64_t)blockIdx.x * chunk;
@@ -120,7 +121,7 @@ k_score_decode(const uint4* __restrict__ q_idx, const float* __restrict__ w, con
     if (kHist) __syncthreads();
 
     if (b0 < b_valid) {
-        const uint8_t* prow = reinterpret_cast<const uint8_t*>(pooled) + (int64_t)s * (kv_capacity / kBlock) * 128;
+        const uint8_t* prow = reinterpret_cast<const uint8_t*>(pooled) + (int64_t)s * (kv_capacity / bs) * 128;
         const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(s_stage);
         const int n_tiles = (int)((b_valid - b0 + kTile - 1) / kTile);
         // stage tile `tl` into slot tl % kStages: 1,024 chunks of 16 B, 4 per thread
@@ -204,17 +205,18 @@ k_score_decode(const uint4* __restrict__ q_idx, const float* __restrict__ w, con
     __threadfence();
     if (sel_idx) {
         // the row's last CTA selects the whole row in shared memory (n_c <= kRowSmemBlocks)
-        select_row_in_smem(S, reinterpret_cast<unsigned*>(s_stage), srow, (int)n_c, cc->hist1,
-                           sel_idx + (int64_t)i * kTopK, sel_cnt + i);
+        select_row_in_smem(S, reinterpret_cast<unsigned*>(s_stage), srow, (int)n_c, top_k, cc->hist1,
+                           sel_idx + (int64_t)i * kSelCap, sel_cnt + i);
         return;
     }
-    finish_digit1(cc, n_c, S.warp);
+    finish_digit1(cc, n_c, top_k, S.warp);
 }
 
 cudaError_t launch_score_decode(const qsa_dims& d, const void* q_idx, const float* w, const void* pooled,
                                 const int32_t* q_seq, const int32_t* q_pos, int32_t row0, int32_t n_rows,
                                 int64_t max_blocks, float* scores, int64_t ld, int chunk, TopkCtrl* ctrl,
-                                int32_t* sel_idx, int32_t* sel_cnt, unsigned* status, cudaStream_t st, bool pdl)
+                                int32_t* sel_idx, int32_t* sel_cnt, unsigned* status, cudaStream_t st, bool pdl,
+                                int pos_stride)
 {
     if (sel_idx && (!ctrl || max_blocks > kRowSmemBlocks)) return cudaErrorInvalidValue;
     if (n_rows <= 0 || max_blocks <= 0) return cudaSuccess;
@@ -234,7 +236,7 @@ cudaError_t launch_score_decode(const qsa_dims& d, const void* q_idx, const floa
     }
     return launch_k(ctrl ? k_score_decode<true> : k_score_decode<false>, grid, dim3(256), kStageBytes, st, pdl,
                     (const uint4*)q_idx, w, (const uint4*)pooled, q_seq, q_pos, row0, d.batch, d.kv_capacity,
-                    max_blocks, scores, ld, chunk, ctrl, sel_idx, sel_cnt, status);
+                    max_blocks, scores, ld, chunk, ctrl, sel_idx, sel_cnt, status, pos_stride, d.block_size, d.top_k);
 }
 
 }  // namespace qsa

@@ -92,18 +92,18 @@ __device__ __forceinline__ void resolve_digit(TopkCtrl* ctrl, const unsigned* hi
     }
 }
 
-// Candidates of query row: n_c(t) = floor((t+1)/4), cut at max_blocks; 0 for an invalid position.
-__device__ __forceinline__ int64_t candidate_blocks(int t, int64_t kv_capacity, int64_t max_blocks)
+// Candidates of query row: n_c(t) = floor((t+1)/bs), cut at max_blocks; 0 for an invalid position.
+__device__ __forceinline__ int64_t candidate_blocks(int t, int64_t kv_capacity, int64_t max_blocks, int bs)
 {
     if (t < 0 || (int64_t)t >= kv_capacity) return 0;
-    const int64_t n_c = ((int64_t)t + 1) / kBlock;
+    const int64_t n_c = ((int64_t)t + 1) / bs;
     return n_c < max_blocks ? n_c : max_blocks;
 }
 
 // Completion of digit 1 (run by the last CTA of the first histogram pass).
-__device__ __forceinline__ void finish_digit1(TopkCtrl* ctrl, int64_t n_c, unsigned* s_warp)
+__device__ __forceinline__ void finish_digit1(TopkCtrl* ctrl, int64_t n_c, int top_k, unsigned* s_warp)
 {
-    if (n_c <= kTopK) {
+    if (n_c <= top_k) {
         if (threadIdx.x == 0) {
             ctrl->n_cand = (int)n_c;
             ctrl->mode = kSelAll;
@@ -111,7 +111,7 @@ __device__ __forceinline__ void finish_digit1(TopkCtrl* ctrl, int64_t n_c, unsig
         return;
     }
     if (threadIdx.x == 0) ctrl->n_cand = (int)n_c;
-    resolve_digit<kBins1 / 256>(ctrl, ctrl->hist1, 12, false, 0u, 0, kTopK, s_warp);
+    resolve_digit<kBins1 / 256>(ctrl, ctrl->hist1, 12, false, 0u, 0, top_k, s_warp);
 }
 
 }  // namespace qsa

@@ -16,7 +16,7 @@ constexpr int kMaxTieRank = 1024;               // keys equal at the cut ranked 
 // 16-byte aligned: hist doubles as scratch for 64-bit sort keys.
 struct alignas(16) FinishSmem {
     unsigned hist[kBins2];
-    int list[kTopK];
+    int list[kSelCap];
     unsigned warp[8];
     int cnt[8];
     int n_list;
@@ -121,7 +121,7 @@ __device__ __forceinline__ void block_sort_512(T* a, T* b)
     T* src = b;
     T* dst = a;
 #pragma unroll 1
-    for (int L = 64; L < kTopK; L <<= 1) {
+    for (int L = 64; L < kSelCap; L <<= 1) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int p = tid + 256 * h;
@@ -159,7 +159,7 @@ __device__ __forceinline__ void take_top_sorted(FinishSmem& S, const unsigned lo
 {
     const int tid = threadIdx.x;
     unsigned long long* a = reinterpret_cast<unsigned long long*>(S.hist);
-    unsigned long long* b = a + kTopK;
+    unsigned long long* b = a + kSelCap;
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
         const int j = tid + 256 * k;
@@ -169,9 +169,9 @@ __device__ __forceinline__ void take_top_sorted(FinishSmem& S, const unsigned lo
     __syncthreads();
     block_sort_512<unsigned long long>(a, b);
     const int base = S.n_list;
-    for (int j = tid; j < need && base + j < kTopK; j += 256) S.list[base + j] = (int)(unsigned)a[j];
+    for (int j = tid; j < need && base + j < kSelCap; j += 256) S.list[base + j] = (int)(unsigned)a[j];
     __syncthreads();
-    if (tid == 0) S.n_list = min(base + need, kTopK);
+    if (tid == 0) S.n_list = min(base + need, kSelCap);
     __syncthreads();
 }
 
@@ -268,7 +268,7 @@ __device__ __forceinline__ bool take_by_cut(FinishSmem& S, const unsigned long l
 #pragma unroll
     for (int k = 0; k < kPerThreadCand; ++k)
         if (take_mask >> k & 1u) {
-            if (slot < kTopK) S.list[slot] = (int)(unsigned)cr[k];
+            if (slot < kSelCap) S.list[slot] = (int)(unsigned)cr[k];
             ++slot;
         }
     __syncthreads();
@@ -280,7 +280,7 @@ __device__ __forceinline__ bool take_by_cut(FinishSmem& S, const unsigned long l
 // Ordered selection of the top `need` keys of a score row in global memory
 // (keys whose top 12 bits exceed `p12` are all taken; among those equal to it the
 // top `need12`), written to S.list in ascending block order.  With `from_digit1`
-// the whole row is ranked (p12 and need12 are ignored; need12 = top_k).
+// the whole row is ranked for its top `need12` (p12 is ignored).
 __device__ inline void select_by_rescan(FinishSmem& S, const float* srow, int64_t n_c, bool from_digit1, unsigned p12,
                                  int need12)
 {
@@ -289,7 +289,6 @@ __device__ inline void select_by_rescan(FinishSmem& S, const float* srow, int64_
     unsigned cut;
     bool whole = false;
     if (from_digit1) {
-        need = kTopK;
         clear_hist(S, kBins1);
         for (int64_t b = tid; b < n_c; b += 256) atomicAdd(&S.hist[orderable_key(__ldcg(srow + b)) >> 20], 1u);
         __syncthreads();
@@ -338,12 +337,12 @@ __device__ inline void select_by_rescan(FinishSmem& S, const float* srow, int64_
         const bool take = valid && (key > cut || (eq && (whole || eq_seen + eq_rank < need)));
         int n_take;
         const int rank = block_rank_256(take, S.cnt, &n_take);
-        if (take && taken + rank < kTopK) S.list[taken + rank] = (int)b;
+        if (take && taken + rank < kSelCap) S.list[taken + rank] = (int)b;
         taken += n_take;
         eq_seen += eq_total;
     }
     __syncthreads();
-    if (tid == 0) S.n_list = taken < kTopK ? taken : kTopK;
+    if (tid == 0) S.n_list = taken < kSelCap ? taken : kSelCap;
     __syncthreads();
 }
 
@@ -361,12 +360,12 @@ constexpr int kRowSmemWords = kRowSmemBlocks + kRowSmemBlocks / 16;
 
 __device__ __forceinline__ int row_pos(int b) { return b + 4 * (b >> 6); }
 
-__device__ inline void select_row_in_smem(FinishSmem& S, unsigned* keys, const float* srow, int n_c,
+__device__ inline void select_row_in_smem(FinishSmem& S, unsigned* keys, const float* srow, int n_c, int top_k,
                                           const unsigned* hist1, int32_t* out, int32_t* cnt_out)
 {
     const int tid = threadIdx.x;
-    if (n_c <= kTopK) {
-        for (int k = tid; k < kTopK; k += 256) out[k] = k < n_c ? k : -1;
+    if (n_c <= top_k) {
+        for (int k = tid; k < kSelCap; k += 256) out[k] = k < n_c ? k : -1;
         if (tid == 0) *cnt_out = n_c;
         return;
     }
@@ -398,7 +397,7 @@ __device__ inline void select_row_in_smem(FinishSmem& S, unsigned* keys, const f
     __syncthreads();
     const uint4* mine = reinterpret_cast<const uint4*>(keys + row_pos(64 * tid));
     // digit 1 (bits 31..20)
-    resolve_smem<kBins1 / 256>(S, kTopK);
+    resolve_smem<kBins1 / 256>(S, top_k);
     unsigned cut = S.res_digit << 20;
     int need = S.res_need;
     bool whole = S.res_count == (unsigned)need;
@@ -462,14 +461,14 @@ __device__ inline void select_row_in_smem(FinishSmem& S, unsigned* keys, const f
         for (int e = 0; e < 4; ++e) {
             const bool is_eq = kv[e] == cut && eq_left > 0;
             if (kv[e] > cut || is_eq) {
-                if (slot < kTopK) out[slot] = 64 * tid + 4 * q + e;
+                if (slot < kSelCap) out[slot] = 64 * tid + 4 * q + e;
                 ++slot;
             }
             eq_left -= is_eq ? 1 : 0;
         }
     }
-    for (int k = (int)n_taken + tid; k < kTopK; k += 256) out[k] = -1;
-    if (tid == 0) *cnt_out = (int)min(n_taken, (unsigned)kTopK);
+    for (int k = (int)n_taken + tid; k < kSelCap; k += 256) out[k] = -1;
+    if (tid == 0) *cnt_out = (int)min(n_taken, (unsigned)top_k);
 }
 
 }  // namespace qsa

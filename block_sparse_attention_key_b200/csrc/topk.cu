@@ -27,7 +27,7 @@ constexpr int kPerThreadLoad = 16;  // score values each collecting thread holds
 // First histogram pass for score rows that come from the caller (qsa_topk_blocks).
 __global__ void __launch_bounds__(256)
 k_topk_pass1(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ q_pos, int32_t row0,
-             int64_t kv_capacity, int64_t max_blocks, int chunk, TopkCtrl* __restrict__ ctrl)
+             int64_t kv_capacity, int64_t max_blocks, int bs, int top_k, int chunk, TopkCtrl* __restrict__ ctrl)
 {
     __shared__ unsigned s_hist[kBins1];
     __shared__ unsigned s_warp[8];
@@ -37,7 +37,7 @@ k_topk_pass1(const float* __restrict__ scores, int64_t ld, const int32_t* __rest
     const int tid = threadIdx.x;
     const int r = blockIdx.y;
     TopkCtrl* c = ctrl + r;
-    const int64_t n_c = candidate_blocks(q_pos[row0 + r], kv_capacity, max_blocks);
+    const int64_t n_c = candidate_blocks(q_pos[row0 + r], kv_capacity, max_blocks, bs);
     const int64_t b0 = (int64_t)blockIdx.x * chunk;
     const int64_t b1 = min(b0 + (int64_t)chunk, n_c);
     const float* srow = scores + (int64_t)r * ld;
@@ -55,15 +55,15 @@ k_topk_pass1(const float* __restrict__ scores, int64_t ld, const int32_t* __rest
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    finish_digit1(c, n_c, s_warp);
+    finish_digit1(c, n_c, top_k, s_warp);
 }
 
 // Collect winners (above the boundary bin) and candidates (inside it); the last
 // CTA of a row settles the selection and writes the ascending list.
 __global__ void __launch_bounds__(256)
-k_topk_collect(const float* __restrict__ scores, int64_t ld, int32_t row0, int chunk, TopkCtrl* __restrict__ ctrl,
-               unsigned long long* __restrict__ cand, int32_t* __restrict__ tmp, int32_t* __restrict__ sel_idx,
-               int32_t* __restrict__ sel_cnt, unsigned* status)
+k_topk_collect(const float* __restrict__ scores, int64_t ld, int32_t row0, int chunk, int top_k,
+               TopkCtrl* __restrict__ ctrl, unsigned long long* __restrict__ cand, int32_t* __restrict__ tmp,
+               int32_t* __restrict__ sel_idx, int32_t* __restrict__ sel_cnt, unsigned* status)
 {
     __shared__ FinishSmem S;
     __shared__ int s_base[2];
@@ -81,7 +81,7 @@ k_topk_collect(const float* __restrict__ scores, int64_t ld, int32_t row0, int c
     const int need1 = c->need;               // blocks still wanted from that bin
     const bool crowded = c->bin_count > (unsigned)kCandCap;
     const float* srow = scores + (int64_t)r * ld;
-    int32_t* win = tmp + (int64_t)r * kTopK;
+    int32_t* win = tmp + (int64_t)r * kSelCap;
     unsigned long long* cl = cand + (int64_t)r * kCandCap;
 
     if (mode != kSelAll) {
@@ -135,7 +135,7 @@ k_topk_collect(const float* __restrict__ scores, int64_t ld, int32_t row0, int c
             for (int k = 0; k < kPer; ++k) {
                 const int64_t b = base + tid + 256 * k;
                 if (wmask >> k & 1u) {
-                    if (wslot < kTopK) win[wslot] = (int32_t)b;
+                    if (wslot < kSelCap) win[wslot] = (int32_t)b;
                     else set_status(status, QSA_DEV_BAD_SEL);
                     ++wslot;
                 }
@@ -155,8 +155,8 @@ k_topk_collect(const float* __restrict__ scores, int64_t ld, int32_t row0, int c
     if (!s_last) return;
     __threadfence();
 
-    const int cnt = (int)min((int64_t)kTopK, n_c);
-    for (int k = tid; k < kTopK; k += 256) S.list[k] = INT_MAX;
+    const int cnt = (int)min((int64_t)top_k, n_c);
+    for (int k = tid; k < kSelCap; k += 256) S.list[k] = INT_MAX;
     if (tid == 0) S.n_list = 0;
     __syncthreads();
 
@@ -165,7 +165,7 @@ k_topk_collect(const float* __restrict__ scores, int64_t ld, int32_t row0, int c
         for (int k = tid; k < cnt; k += 256) S.list[k] = k;
         sorted = true;
     } else if (mode == kSelPrefix) {
-        for (int k = tid; k < kTopK; k += 256) S.list[k] = __ldcg(win + k);
+        for (int k = tid; k < cnt; k += 256) S.list[k] = __ldcg(win + k);
     } else if (crowded) {
         select_by_rescan(S, srow, n_c, false, b1, need1);
         sorted = true;
@@ -178,17 +178,17 @@ k_topk_collect(const float* __restrict__ scores, int64_t ld, int32_t row0, int c
             const int j = tid + 256 * k;
             cr[k] = j < nc ? __ldcg(cl + j) : 0ull;
         }
-        const int n_win = (int)min(__ldcg(&c->nsel), (unsigned)kTopK);
+        const int n_win = (int)min(__ldcg(&c->nsel), (unsigned)top_k);
         for (int k = tid; k < n_win; k += 256) S.list[k] = __ldcg(win + k);
         if (tid == 0) S.n_list = n_win;
         __syncthreads();
-        if (nc <= kTopK) {
+        if (nc <= kSelCap) {  // a sort of at most kSelCap entries
             // few candidates: sort them by (key desc, block asc) and take the first need1
             take_top_sorted(S, cr, nc, need1);
         } else {
             const Cut cut = resolve_cut_regs(S, cr, nc, need1, false, b1);
             if (!take_by_cut(S, cr, nc, cut)) {
-                for (int k = tid; k < kTopK; k += 256) S.list[k] = INT_MAX;
+                for (int k = tid; k < kSelCap; k += 256) S.list[k] = INT_MAX;
                 __syncthreads();
                 select_by_rescan(S, srow, n_c, false, b1, need1);
                 sorted = true;
@@ -197,13 +197,14 @@ k_topk_collect(const float* __restrict__ scores, int64_t ld, int32_t row0, int c
     }
     __syncthreads();
     if (!sorted) sort_list_512(S);
-    int32_t* out = sel_idx + (int64_t)i * kTopK;
-    for (int k = tid; k < kTopK; k += 256) out[k] = k < cnt ? S.list[k] : -1;
+    int32_t* out = sel_idx + (int64_t)i * kSelCap;
+    for (int k = tid; k < kSelCap; k += 256) out[k] = k < cnt ? S.list[k] : -1;
     if (tid == 0) sel_cnt[i] = cnt;
 }
 
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, int32_t row0, int32_t n_rows,
-                        int64_t max_blocks, int64_t kv_capacity, int chunk, int n_chunks, TopkCtrl* ctrl,
+                        int64_t max_blocks, int64_t kv_capacity, int bs, int top_k, int chunk, int n_chunks,
+                        TopkCtrl* ctrl,
                         unsigned long long* cand, int32_t* tmp, int32_t* sel_idx, int32_t* sel_cnt, bool hist_done,
                         unsigned* status, cudaStream_t st, bool pdl)
 {
@@ -211,11 +212,11 @@ cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, i
     dim3 grid((unsigned)(n_chunks > 0 ? n_chunks : 1), (unsigned)n_rows);
     if (!hist_done) {
         const cudaError_t e = launch_k(k_topk_pass1, grid, dim3(256), 0, st, false, scores, ld, q_pos, row0,
-                                       kv_capacity, max_blocks, chunk, ctrl);
+                                       kv_capacity, max_blocks, bs, top_k, chunk, ctrl);
         if (e != cudaSuccess) return e;
     }
-    return launch_k(k_topk_collect, grid, dim3(256), 0, st, hist_done ? pdl : true, scores, ld, row0, chunk, ctrl,
-                    cand, tmp, sel_idx, sel_cnt, status);
+    return launch_k(k_topk_collect, grid, dim3(256), 0, st, hist_done ? pdl : true, scores, ld, row0, chunk, top_k,
+                    ctrl, cand, tmp, sel_idx, sel_cnt, status);
 }
 
 }  // namespace qsa

@@ -12,6 +12,8 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libqsa.so")
 
+QSA_SEL_CAP = 512
+
 QSA_OK = 0
 QSA_ERR_INVALID_ARG = -1
 QSA_ERR_WORKSPACE_TOO_SMALL = -2
@@ -25,15 +27,20 @@ QSA_DEV_BAD_LEN = 0x8
 QSA_DEV_BAD_SEL = 0x10
 QSA_DEV_TOO_MANY_NEW = 0x20
 QSA_DEV_TIMEOUT = 0x40
+QSA_DEV_BAD_PAGE = 0x80
 
 QSA_MODE_DECODE = 0
 QSA_MODE_PREFILL = 1
+QSA_MODE_MIXED = 2
 
 EXPORTED = (
     "qsa_workspace_bytes", "qsa_workspace_init", "qsa_read_device_status", "qsa_status_string",
     "qsa_pool_block_keys", "qsa_index_scores", "qsa_topk_blocks", "qsa_sparse_attn", "qsa_forward",
-    "qsa_sparse_attn_noalloc",
+    "qsa_sparse_attn_noalloc", "qsa_sparse_attn_ex", "qsa_select_blocks",
+    "qsa_cp_workspace_bytes", "qsa_cp_select_keys", "qsa_cp_merge_keys", "qsa_cp_attn_partial", "qsa_cp_combine",
 )
+
+CP_PART_ROW = 132  # floats per (query, head) partial of a context shard
 
 
 class QsaError(RuntimeError):
@@ -59,6 +66,18 @@ class qsa_forward_args(ctypes.Structure):
         ("q_seq", ctypes.c_void_p), ("q_pos", ctypes.c_void_p), ("n_q", ctypes.c_int32),
         ("max_new_tokens", ctypes.c_int32), ("max_blocks", ctypes.c_int64), ("mode", ctypes.c_int32),
         ("sel_idx", ctypes.c_void_p), ("sel_cnt", ctypes.c_void_p), ("out", ctypes.c_void_p),
+        ("group_q", ctypes.c_int32), ("page_table", ctypes.c_void_p), ("page_tokens", ctypes.c_int32),
+        ("n_pages", ctypes.c_int64), ("n_decode", ctypes.c_int32),
+    ]
+
+
+class qsa_attn_args(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+        ("q_seq", ctypes.c_void_p), ("q_pos", ctypes.c_void_p), ("sel_idx", ctypes.c_void_p),
+        ("sel_cnt", ctypes.c_void_p), ("n_q", ctypes.c_int32), ("group_q", ctypes.c_int32),
+        ("page_table", ctypes.c_void_p), ("page_tokens", ctypes.c_int32), ("n_pages", ctypes.c_int64),
+        ("out", ctypes.c_void_p),
     ]
 
 
@@ -87,8 +106,16 @@ def load(path=LIB_PATH):
     L.qsa_sparse_attn.argtypes = [D, P, P, P, P, P, P, P, I32, P, P, SZ, P]
     L.qsa_forward.argtypes = [D, ctypes.POINTER(qsa_forward_args), P, SZ, P]
     L.qsa_sparse_attn_noalloc.argtypes = [D, P, P, P, P, P, P, P, I32, P, P]
+    L.qsa_sparse_attn_ex.argtypes = [D, ctypes.POINTER(qsa_attn_args), P, SZ, P]
+    L.qsa_select_blocks.argtypes = [D, P, P, P, P, P, I32, I64, I32, P, P, P, SZ, P]
+    L.qsa_cp_workspace_bytes.argtypes = [D, I32]
+    L.qsa_cp_workspace_bytes.restype = SZ
+    L.qsa_cp_select_keys.argtypes = [D, P, P, P, P, P, I32, I64, P, P, P, SZ, P]
+    L.qsa_cp_merge_keys.argtypes = [D, I32, P, P, I32, I64, P, P, P, P, P]
+    L.qsa_cp_attn_partial.argtypes = [D, P, P, P, P, P, I32, I64, P, P, P, P, SZ, P]
+    L.qsa_cp_combine.argtypes = [D, I32, P, I32, P, P]
     for name in EXPORTED:
-        if name not in ("qsa_workspace_bytes", "qsa_status_string"):
+        if name not in ("qsa_workspace_bytes", "qsa_status_string", "qsa_cp_workspace_bytes"):
             getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -165,6 +192,14 @@ def qsa_topk_blocks(dims, scores, ld_scores, q_pos, n_q, max_blocks, sel_idx, se
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def qsa_select_blocks(dims, q_idx, w, pooled, q_seq, q_pos, n_q, max_blocks, mode, sel_idx, sel_cnt, workspace,
+                      stream=None):
+    _check("qsa_select_blocks", load().qsa_select_blocks(
+        ctypes.byref(dims), _ptr(q_idx), _ptr(w), _ptr(pooled), _ptr(q_seq), _ptr(q_pos), n_q, max_blocks, mode,
+        _ptr(sel_idx), _ptr(sel_cnt), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+
+
 def qsa_sparse_attn(dims, q, k_cache, v_cache, q_seq, q_pos, sel_idx, sel_cnt, n_q, out, workspace, stream=None):
     _check("qsa_sparse_attn", load().qsa_sparse_attn(
         ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(q_seq), _ptr(q_pos), _ptr(sel_idx),
@@ -180,10 +215,54 @@ def qsa_sparse_attn_noalloc(dims, q, k_cache, v_cache, q_seq, q_pos, sel_idx, se
         _ptr(sel_cnt), n_q, _ptr(out), _stream(stream)))
 
 
+def qsa_sparse_attn_ex(dims, *, q, k_cache, v_cache, q_seq, q_pos, sel_idx, sel_cnt, n_q, out, workspace,
+                       group_q=1, page_table=None, page_tokens=0, n_pages=0, stream=None):
+    args = qsa_attn_args(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(q_seq), _ptr(q_pos), _ptr(sel_idx),
+                         _ptr(sel_cnt), n_q, group_q, _ptr(page_table), page_tokens, n_pages, _ptr(out))
+    _check("qsa_sparse_attn_ex", load().qsa_sparse_attn_ex(ctypes.byref(dims), ctypes.byref(args), _ptr(workspace),
+                                                           workspace.numel() * workspace.element_size(),
+                                                           _stream(stream)))
+
+
 def qsa_forward(dims, *, q, k_cache, v_cache, idx_k, pooled, q_idx, w, len_before, len_after, q_seq, q_pos,
-                n_q, max_new_tokens, max_blocks, mode, out, workspace, sel_idx=None, sel_cnt=None, stream=None):
+                n_q, max_new_tokens, max_blocks, mode, out, workspace, sel_idx=None, sel_cnt=None, group_q=0,
+                page_table=None, page_tokens=0, n_pages=0, n_decode=0, stream=None):
     args = qsa_forward_args(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(idx_k), _ptr(pooled), _ptr(q_idx),
                             _ptr(w), _ptr(len_before), _ptr(len_after), _ptr(q_seq), _ptr(q_pos), n_q,
-                            max_new_tokens, max_blocks, mode, _ptr(sel_idx), _ptr(sel_cnt), _ptr(out))
+                            max_new_tokens, max_blocks, mode, _ptr(sel_idx), _ptr(sel_cnt), _ptr(out), group_q,
+                            _ptr(page_table), page_tokens, n_pages, n_decode)
     _check("qsa_forward", load().qsa_forward(ctypes.byref(dims), ctypes.byref(args), _ptr(workspace),
                                              workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+# ---------------------------------------------------------------- context parallelism (see include/qsa.h)
+
+def qsa_cp_workspace_bytes(shard_dims, n_q):
+    return int(load().qsa_cp_workspace_bytes(ctypes.byref(shard_dims), n_q))
+
+
+def qsa_cp_select_keys(shard_dims, q_idx, w, pooled_shard, q_seq, q_pos, n_q, blk_lo, keys, key_cnt, workspace,
+                       stream=None):
+    _check("qsa_cp_select_keys", load().qsa_cp_select_keys(
+        ctypes.byref(shard_dims), _ptr(q_idx), _ptr(w), _ptr(pooled_shard), _ptr(q_seq), _ptr(q_pos), n_q, blk_lo,
+        _ptr(keys), _ptr(key_cnt), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def qsa_cp_merge_keys(shard_dims, n_ranks, keys_all, cnt_all, n_q, blk_lo, sel_local, cnt_local, sel_global=None,
+                      cnt_global=None, stream=None):
+    _check("qsa_cp_merge_keys", load().qsa_cp_merge_keys(
+        ctypes.byref(shard_dims), n_ranks, _ptr(keys_all), _ptr(cnt_all), n_q, blk_lo, _ptr(sel_local),
+        _ptr(cnt_local), _ptr(sel_global), _ptr(cnt_global), _stream(stream)))
+
+
+def qsa_cp_attn_partial(shard_dims, q, k_shard, v_shard, q_seq, q_pos, n_q, blk_lo, sel_local, cnt_local, part,
+                        workspace, stream=None):
+    _check("qsa_cp_attn_partial", load().qsa_cp_attn_partial(
+        ctypes.byref(shard_dims), _ptr(q), _ptr(k_shard), _ptr(v_shard), _ptr(q_seq), _ptr(q_pos), n_q, blk_lo,
+        _ptr(sel_local), _ptr(cnt_local), _ptr(part), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+
+
+def qsa_cp_combine(dims, n_ranks, parts_all, n_q, out, stream=None):
+    _check("qsa_cp_combine", load().qsa_cp_combine(ctypes.byref(dims), n_ranks, _ptr(parts_all), n_q, _ptr(out),
+                                                   _stream(stream)))

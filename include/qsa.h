@@ -36,7 +36,12 @@
  *   traps, asserts or waits without bound.
  * - Outputs never alias inputs; `pooled` is the only in-out tensor.
  *
- * Layouts (B = batch, T = kv_capacity, Nb = T/4 pooled blocks, n_q = queries):
+ * Block size and budget: the published setting is 4-token blocks and 512 blocks
+ * per query; dims.block_size may be any power of two up to 16 (1 = per-token
+ * selection) and dims.top_k any value in [1, QSA_SEL_CAP].  Below, 4 and 512 stand
+ * for block_size and top_k, and n_c(t) = floor((t+1)/block_size).
+ *
+ * Layouts (B = batch, T = kv_capacity, Nb = T/block_size pooled blocks, n_q = queries):
  *   q        bf16 [n_q][n_q_heads][head_dim]
  *   k_cache  bf16 [B][n_kv_heads][T][head_dim]   (head-major: one block of one
  *   v_cache  bf16 [B][n_kv_heads][T][head_dim]    head is 1 KiB contiguous)
@@ -46,7 +51,7 @@
  *   w        f32  [n_q][n_idx_heads]
  *   q_seq    i32  [n_q]   sequence of each query, in [0, B)
  *   q_pos    i32  [n_q]   0-based position of each query, in [0, T)
- *   sel_idx  i32  [n_q][top_k]  ascending selected blocks, padded with -1
+ *   sel_idx  i32  [n_q][QSA_SEL_CAP]  ascending selected blocks, padded with -1
  *   sel_cnt  i32  [n_q]   min(top_k, n_c(t))
  *   out      bf16 [n_q][n_q_heads][head_dim]
  * Query head h reads KV head h / (n_q_heads / n_kv_heads).
@@ -60,6 +65,9 @@
 #ifdef __cplusplus
 extern "C" {
 #endif
+
+/* Capacity of one query's selection: the row stride of every sel_idx array. */
+#define QSA_SEL_CAP 512
 
 /* ---- status codes (return values) ---- */
 #define QSA_OK                       0
@@ -76,10 +84,15 @@ extern "C" {
 #define QSA_DEV_BAD_SEL        0x10u /* sel_idx entry outside [0, n_c(t)) or sel_cnt > top_k: skipped */
 #define QSA_DEV_TOO_MANY_NEW   0x20u /* len_after - len_before > max_new_tokens: rest not pooled */
 #define QSA_DEV_TIMEOUT        0x40u /* a bounded in-kernel wait gave up: results of that call are invalid */
+#define QSA_DEV_BAD_PAGE       0x80u /* page-table entry < 0 for an attended token: its block skipped */
 
 /* ---- forward modes ---- */
 #define QSA_MODE_DECODE  0  /* few queries per sequence: split-K attention, multi-CTA select */
-#define QSA_MODE_PREFILL 1  /* a chunk of queries of ONE sequence (all q_seq equal) */
+#define QSA_MODE_PREFILL 1  /* chunks of many queries per sequence (ragged: several sequences per
+                                call; keep each sequence's rows contiguous, since every 128-row
+                                tile makes one scoring pass per distinct sequence it holds) */
+#define QSA_MODE_MIXED   2  /* a serving batch: rows [0, n_decode) decode queries, the rest prefill
+                                chunks; one call, one attention launch over every row */
 
 typedef struct qsa_dims {
     int32_t batch;        /* B, number of sequences (caches) */
@@ -88,19 +101,22 @@ typedef struct qsa_dims {
     int32_t head_dim;     /* must be 128 */
     int32_t n_idx_heads;  /* indexer heads, must be 4 */
     int32_t idx_dim;      /* indexer head dim, must be 64 */
-    int32_t block_size;   /* micro-block size, must be 4 */
-    int32_t top_k;        /* blocks kept per query, must be 512 */
-    int64_t kv_capacity;  /* T, tokens per sequence cache; multiple of 4, < 2^31 */
+    int32_t block_size;   /* micro-block size: 1, 2, 4 (published), 8 or 16 */
+    int32_t top_k;        /* blocks kept per query: 1 .. QSA_SEL_CAP (512 published) */
+    int64_t kv_capacity;  /* T, tokens per sequence cache; multiple of block_size, < 2^31 */
     float softmax_scale;  /* <= 0 selects 1/sqrt(head_dim) */
 } qsa_dims;
 
 /* Workspace bytes qsa_forward needs for n_q queries whose complete causal blocks
- * never exceed max_blocks, in `mode`.  The standalone qsa_topk_blocks and
+ * never exceed max_blocks, in `mode` (QSA_MODE_MIXED: any split of n_q into decode
+ * and prefill rows).  The standalone qsa_topk_blocks and
  * qsa_sparse_attn need at most the QSA_MODE_DECODE figure for the same sizes.
  * Returns 0 on invalid arguments. */
 size_t qsa_workspace_bytes(const qsa_dims* dims, int32_t n_q, int64_t max_blocks, int32_t mode);
 
-/* Zero the workspace's status word.  Call once after allocating a workspace. */
+/* Zero the whole workspace (its status word and the attention's split counters,
+ * which every call leaves at zero again).  Call once after allocating a workspace,
+ * before its first use. */
 int qsa_workspace_init(void* workspace, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, copy the device status word (QSA_DEV_* bits, 0 = clean)
@@ -141,6 +157,18 @@ int qsa_topk_blocks(const qsa_dims* dims, const float* scores, int64_t ld_scores
                     int32_t* sel_idx, int32_t* sel_cnt, void* workspace, size_t ws_bytes,
                     void* stream);
 
+/* Steps 2 and 3 together: scores and the top-k selection of n_q queries, run the
+ * way qsa_forward runs them in `mode` (after its pooling step): QSA_MODE_DECODE
+ * streams every row's scores through workspace score rows (rows of up to 16,384
+ * blocks are selected inside the scoring kernel); QSA_MODE_PREFILL (chunks of
+ * queries, ideally contiguous per sequence) scores on the tensor cores and keeps per row only the blocks
+ * that can still reach its top 512, so no n_q x n_blocks score matrix exists.
+ * Writes sel_idx / sel_cnt as qsa_topk_blocks does.
+ * Needs qsa_workspace_bytes(dims, n_q, max_blocks, mode) bytes. */
+int qsa_select_blocks(const qsa_dims* dims, const void* q_idx, const float* w, const void* pooled,
+                      const int32_t* q_seq, const int32_t* q_pos, int32_t n_q, int64_t max_blocks, int32_t mode,
+                      int32_t* sel_idx, int32_t* sel_cnt, void* workspace, size_t ws_bytes, void* stream);
+
 /* Step 4 — gathered GQA attention over the selected blocks plus the query's
  * partial block:  out[i][h] = sum_j softmax_j(scale * q[i][h].K[s][g][j]) V[s][g][j],
  * g = h / group, j over the 4 tokens of every selected block and the tokens
@@ -166,13 +194,56 @@ int qsa_sparse_attn(const qsa_dims* dims, const void* q, const void* k_cache, co
  * The first call on each device, with that device current, looks the array's
  * device address up (cudaGetSymbolAddress), and so does every later call made
  * outside stream capture (a device reset may move the array); make that first
- * call before any stream capture.  All calls share the array: counters are cleared at the start
- * of each call, and calls whose executions overlap on the GPU race on it.  No
+ * call before any stream capture.  All calls share the array: counters are
+ * cleared at the start of each call, and calls whose executions overlap on the
+ * GPU race on it.  No
  * device status word: out-of-range indices are skipped but not reported.
  * Nothing in this call allocates memory. */
 int qsa_sparse_attn_noalloc(const qsa_dims* dims, const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,
                             const int32_t* sel_cnt, int32_t n_q, void* out, void* stream);
+
+/* Step 4, general form: draft queries that share one selection, and paged K/V.
+ *
+ * Shared selections (keieiax.jp glossary "Qwen Sparse Attention", FAQ on
+ * multi-token prediction: the top index is reused between speculative steps):
+ * with group_q = k >= 2, queries [k*g, k*g + k) form group g, the k draft tokens
+ * of one sequence.  They share selection row g (sel_idx[g], sel_cnt[g], made for
+ * the group's first query at t_0 = q_pos[k*g]) and one gather.  Draft query j at
+ * position t_j attends the shared blocks plus every token from 4*floor((t_0+1)/4)
+ * to t_j.  Requirements (else the query is skipped and QSA_DEV_BAD_SEQ or
+ * QSA_DEV_BAD_POS set): same q_seq as the group's first query, and
+ * t_0 <= t_j <= 4*floor((t_0+1)/4) + 7 (the tail spans at most two blocks).
+ * group_q * (n_q_heads / n_kv_heads) <= 32 and n_q a multiple of group_q.
+ * group_q = 1 is qsa_sparse_attn.
+ *
+ * Paged K/V: with page_table != NULL, k_cache and v_cache are page pools
+ * bf16 [n_pages][n_kv_heads][page_tokens][head_dim] and token p of sequence s
+ * lies in page page_table[s][p / page_tokens] (i32 [batch][kv_capacity /
+ * page_tokens], row p % page_tokens).  page_tokens is a multiple of 4 dividing
+ * kv_capacity, so a block never straddles pages.  An attended block whose page
+ * entry is outside [0, n_pages) is skipped and QSA_DEV_BAD_PAGE set.  The indexer
+ * keys and the pooled cache stay dense per sequence.
+ *
+ * Workspace: qsa_workspace_bytes(dims, n_q, 0, QSA_MODE_DECODE) bytes. */
+typedef struct qsa_attn_args {
+    const void* q;              /* bf16 [n_q][n_q_heads][head_dim] */
+    const void* k_cache;        /* dense caches or page pools (see above) */
+    const void* v_cache;
+    const int32_t* q_seq;       /* i32 [n_q] */
+    const int32_t* q_pos;       /* i32 [n_q] */
+    const int32_t* sel_idx;     /* i32 [n_q / group_q][top_k] */
+    const int32_t* sel_cnt;     /* i32 [n_q / group_q] */
+    int32_t n_q;                /* queries */
+    int32_t group_q;            /* queries per shared selection (>= 1) */
+    const int32_t* page_table;  /* NULL: dense caches */
+    int32_t page_tokens;        /* tokens per page (paged only) */
+    int64_t n_pages;            /* pages in each pool (paged only) */
+    void* out;                  /* bf16 [n_q][n_q_heads][head_dim] */
+} qsa_attn_args;
+
+int qsa_sparse_attn_ex(const qsa_dims* dims, const qsa_attn_args* args, void* workspace, size_t ws_bytes,
+                       void* stream);
 
 /* All inputs of one layer call (see the layouts above). */
 typedef struct qsa_forward_args {
@@ -194,6 +265,18 @@ typedef struct qsa_forward_args {
     int32_t* sel_idx;         /* optional out i32 [n_q][top_k] (NULL: kept in workspace) */
     int32_t* sel_cnt;         /* optional out i32 [n_q] */
     void* out;                /* bf16 [n_q][n_q_heads][head_dim] */
+    /* multi-token decode (QSA_MODE_DECODE only; see qsa_sparse_attn_ex): 0 or 1 =
+     * one selection per query; k >= 2: each group of k consecutive draft queries is
+     * scored and selected once, for its first query, with q_idx / w / sel_idx /
+     * sel_cnt holding one row per group, and attends as qsa_sparse_attn_ex says */
+    int32_t group_q;
+    /* paged K/V (see qsa_sparse_attn_ex); page_table NULL = dense caches */
+    const int32_t* page_table;
+    int32_t page_tokens;
+    int64_t n_pages;
+    /* QSA_MODE_MIXED only: rows [0, n_decode) are decode queries, [n_decode, n_q) prefill
+     * chunks (q_idx, w, q_seq, q_pos, sel_idx, sel_cnt, q and out in that row order) */
+    int32_t n_decode;
 } qsa_forward_args;
 
 /* The whole layer: pool the appended blocks, score, select, attend.
@@ -201,6 +284,46 @@ typedef struct qsa_forward_args {
  * n_q x n_keys is ever allocated or built; the library allocates nothing. */
 int qsa_forward(const qsa_dims* dims, const qsa_forward_args* args, void* workspace,
                 size_t ws_bytes, void* stream);
+
+/* ---- context parallelism: one sequence's blocks spread over several GPUs ----
+ *
+ * ai-manual.ru, discussion of llama.cpp PR #30965 (closing note): several GPUs add
+ * memory but add exchange between the cards.  The layer splits exactly along its two
+ * reductions, with two all-gathers between the steps below (made by the caller, e.g.
+ * NCCL over NVLink):
+ *   1. qsa_cp_select_keys: each GPU scores the blocks it holds and keeps its local
+ *      top_k as 64-bit keys (order-preserving score << 32 | ~global block): the
+ *      global top_k (score descending, lower block on ties) is a subset of the union;
+ *   2. all-gather the keys and counts;
+ *   3. qsa_cp_merge_keys: every GPU merges the same union into the same global
+ *      selection and keeps the blocks of its own shard;
+ *   4. qsa_cp_attn_partial: each GPU attends its selected blocks (and the query's
+ *      partial block if the query's last tokens are in its shard) and writes one
+ *      unnormalised partial per (query, head);
+ *   5. all-gather the partials;  6. qsa_cp_combine: the softmax over the union.
+ * A shard is the block range [blk_lo, blk_lo + n_local) of every sequence, held in
+ * the usual layouts with kv_capacity = n_local * block_size tokens (so `shard`
+ * describes the local caches); positions (q_pos) stay global.  Decode-shaped calls
+ * (few queries per sequence).  Keys: u64 [n_q][QSA_SEL_CAP] (unused slots 0),
+ * counts i32 [n_q]; gathered arrays are rank-major ([n_ranks][n_q]...).  Partials:
+ * f32 [n_q][n_q_heads][132] = (max, sum, 2 unused, 128 weighted values), exp2 domain.
+ * Workspace: qsa_cp_workspace_bytes(shard, n_q), initialised with qsa_workspace_init. */
+size_t qsa_cp_workspace_bytes(const qsa_dims* shard, int32_t n_q);
+int qsa_cp_select_keys(const qsa_dims* shard, const void* q_idx, const float* w, const void* pooled_shard,
+                       const int32_t* q_seq, const int32_t* q_pos, int32_t n_q, int64_t blk_lo, uint64_t* keys,
+                       int32_t* key_cnt, void* workspace, size_t ws_bytes, void* stream);
+/* n_ranks <= 8.  sel_local / cnt_local: this shard's blocks of the global selection,
+ * ascending, as shard-local indices (-1 padded); sel_global / cnt_global (optional,
+ * NULL to skip): the whole global selection. */
+int qsa_cp_merge_keys(const qsa_dims* shard, int32_t n_ranks, const uint64_t* keys_all, const int32_t* cnt_all,
+                      int32_t n_q, int64_t blk_lo, int32_t* sel_local, int32_t* cnt_local, int32_t* sel_global,
+                      int32_t* cnt_global, void* stream);
+int qsa_cp_attn_partial(const qsa_dims* shard, const void* q, const void* k_shard, const void* v_shard,
+                        const int32_t* q_seq, const int32_t* q_pos, int32_t n_q, int64_t blk_lo,
+                        const int32_t* sel_local, const int32_t* cnt_local, float* part, void* workspace,
+                        size_t ws_bytes, void* stream);
+int qsa_cp_combine(const qsa_dims* dims, int32_t n_ranks, const float* parts_all, int32_t n_q, void* out,
+                   void* stream);
 
 #ifdef __cplusplus
 }

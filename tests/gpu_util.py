@@ -63,7 +63,7 @@ def run_forward(dw, step, mode=None, ws=None):
     if ws is None or ws.numel() < need:
         ws = new_workspace(need)
     out = torch.empty((T["n_q"], wl.n_q_heads, wl.head_dim), dtype=torch.bfloat16, device="cuda")
-    sel_idx = torch.empty((T["n_q"], wl.top_k), dtype=torch.int32, device="cuda")
+    sel_idx = torch.empty((T["n_q"], qsa.QSA_SEL_CAP), dtype=torch.int32, device="cuda")
     sel_cnt = torch.empty((T["n_q"],), dtype=torch.int32, device="cuda")
     qsa.qsa_forward(dims, q=T["q"], k_cache=dw.k_cache, v_cache=dw.v_cache, idx_k=dw.idx_k, pooled=dw.pooled,
                     q_idx=T["q_idx"], w=T["w"], len_before=T["len_before"], len_after=T["len_after"],

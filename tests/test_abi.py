@@ -61,10 +61,15 @@ def _dims(qsa, **kw):
 def test_workspace_bytes_rejects_bad_dims(qsa):
     ok = qsa.qsa_workspace_bytes(_dims(qsa), 16, 16384, qsa.QSA_MODE_DECODE)
     assert ok > 0
-    bad = [dict(block_size=8), dict(top_k=256), dict(head_dim=64), dict(idx_dim=32), dict(n_idx_heads=2),
-           dict(n_q_heads=30), dict(kv_capacity=65537), dict(batch=0), dict(n_q_heads=64, n_kv_heads=2)]
+    bad = [dict(block_size=3), dict(block_size=0), dict(block_size=32), dict(top_k=0), dict(top_k=513),
+           dict(head_dim=64), dict(idx_dim=32), dict(n_idx_heads=2), dict(n_q_heads=30), dict(kv_capacity=65537),
+           dict(batch=0), dict(n_q_heads=64, n_kv_heads=2), dict(block_size=16, kv_capacity=65544)]
     for kw in bad:
         assert qsa.qsa_workspace_bytes(_dims(qsa, **kw), 16, 16384, 0) == 0, kw
+    # other micro-block sizes and budgets: per-token selection (block 1), coarser blocks, smaller k
+    for kw in [dict(block_size=1), dict(block_size=2), dict(block_size=8), dict(block_size=16), dict(top_k=1),
+               dict(top_k=256), dict(block_size=1, top_k=512)]:
+        assert qsa.qsa_workspace_bytes(_dims(qsa, **kw), 16, 4096, 0) > 0, kw
     assert qsa.qsa_workspace_bytes(_dims(qsa), 16, 16385 + 65536 // 4, 0) == 0   # max_blocks > capacity/4
     assert qsa.qsa_workspace_bytes(_dims(qsa), -1, 16384, 0) == 0
     assert qsa.qsa_workspace_bytes(_dims(qsa), 16, 16384, 7) == 0
@@ -153,9 +158,11 @@ def test_binding_constants_match_the_header(qsa):
     """Every QSA_* value the header defines has the same value in the binding."""
     text = open(os.path.join(ROOT, "include", "qsa.h")).read()
     defs = dict(re.findall(r"^#define\s+(QSA_(?:OK|ERR_\w+|DEV_\w+|MODE_\w+))\s+(-?(?:0x)?[0-9A-Fa-f]+)u?\b", text, re.M))
-    assert len(defs) == 14  # 5 return codes, 7 device status bits, 2 modes
+    assert len(defs) == 16  # 5 return codes, 8 device status bits, 3 modes
     for name, val in defs.items():
         assert getattr(qsa, name) == int(val, 0), name
+    cap = re.search(r"^#define\s+QSA_SEL_CAP\s+(\d+)", text, re.M)
+    assert cap and int(cap.group(1)) == qsa.QSA_SEL_CAP
 
 
 def test_workspace_grows_with_queries_and_blocks(qsa):

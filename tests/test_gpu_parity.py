@@ -379,19 +379,25 @@ def test_prefill_tie_storm_takes_lowest_blocks():
         np.testing.assert_array_equal(sel[r, : cnt[r]], np.arange(cnt[r]))
 
 
-def test_prefill_row_of_another_sequence_is_rejected():
-    wl = W.Workload("pf_badseq", 94, "prefill", 2, 8, 1, 4096, [W.Step([3000, 0], [3000, 0], [0] * 130,
-                                                                      list(range(2870, 3000)), list(range(130)))])
+def test_forward_prefill_ragged_chunks_of_several_sequences():
+    """One prefill call holding chunks of three sequences of different lengths (128-row
+    tiles straddle the chunk boundaries), every row against the oracle."""
+    q_seq = [0] * 100 + [1] * 200 + [2] * 40
+    q_pos = list(range(2000, 2100)) + list(range(5000, 5200)) + list(range(300, 340))
+    wl = W.Workload("pf_ragged", 94, "prefill", 3, 8, 1, 8192,
+                    [W.Step([2000, 5000, 300], [2100, 5200, 340], q_seq, q_pos, list(range(len(q_pos))))])
+    _forward_vs_oracle(wl)
 
-    def mix(q_seq):
-        q_seq = q_seq.clone()
-        q_seq[5] = 1   # tile 0 belongs to sequence 0
-        return q_seq
-    sel, cnt, flags = _prefill_run(wl, q_seq_override=mix)
-    import block_sparse_attention_key_b200 as qsa
-    assert flags & qsa.qsa.QSA_DEV_BAD_SEQ
-    assert cnt[5] == 0 and (sel[5] == -1).all()
-    assert cnt[4] == 512 and cnt[129] == 512
+
+def test_forward_prefill_interleaved_sequences():
+    """Rows of two sequences interleaved row by row: every 128-row tile scores both
+    sequences' pooled keys (one pass each), rows keep their own sequence's blocks."""
+    n = 160
+    q_seq = [r % 2 for r in range(n)]
+    q_pos = [3000 + r // 2 if r % 2 == 0 else 6000 + r // 2 for r in range(n)]
+    wl = W.Workload("pf_interleaved", 93, "prefill", 2, 16, 2, 8192,
+                    [W.Step([3000, 6000], [3000 + n // 2, 6000 + n // 2], q_seq, q_pos, list(range(n)))])
+    _forward_vs_oracle(wl)
 
 
 @pytest.mark.parametrize("cap", [8192, 65536, 131072])
@@ -428,3 +434,30 @@ def test_forward_decode_ties_take_lowest_blocks(cap):
         want = O.select_top_blocks(O.block_scores(q_bits[r], w[r], pooled_bits))
         assert cnt[r] == len(want)
         np.testing.assert_array_equal(sel[r, : cnt[r]], want, err_msg=f"row {r}")
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_select_blocks_entry_point_matches_oracle(mode):
+    """qsa_select_blocks (scores + top-512 alone) in both modes, against the oracle."""
+    import block_sparse_attention_key_b200 as qsa
+    from qsa_synth import device as sdev
+    wl = W.Workload(f"select_only_{mode}", 91, "prefill", 1, 8, 1, 65536, [W._prefill_step(60000, 130)])
+    dw = sdev.DeviceWorkload(wl)
+    gu.pool_history(dw, 0)
+    T = dw.step_tensors(0)
+    n = T["n_q"]
+    dims = gu.dims_of(wl)
+    # the chunk's own tokens must be pooled too: pool the whole appended range first
+    qsa.qsa_pool_block_keys(dims, dw.idx_k, dw.pooled, T["len_before"], T["len_after"], T["max_new_tokens"])
+    ws = gu.new_workspace(qsa.qsa_workspace_bytes(dims, n, T["max_blocks"], mode))
+    sel = torch.empty((n, 512), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((n,), dtype=torch.int32, device="cuda")
+    qsa.qsa_select_blocks(dims, T["q_idx"], T["w"], dw.pooled, T["q_seq"], T["q_pos"], n, T["max_blocks"], mode,
+                          sel, cnt, ws)
+    assert qsa.qsa_read_device_status(ws) == 0
+    gu.check_selection_properties(wl, 0, sel, cnt)
+    wo = O.WorkloadOracle(wl)
+    sel, cnt = sel.cpu().numpy(), cnt.cpu().numpy()
+    for r in [0, 1, 2, 3, 64, 127, 128, 129]:
+        s_want, _ = wo.query(0, r)
+        np.testing.assert_array_equal(sel[r, : cnt[r]], s_want, err_msg=f"row {r}")
