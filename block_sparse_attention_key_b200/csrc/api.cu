@@ -107,7 +107,7 @@ WsLayout plan_workspace(const qsa_dims& d, int32_t n_q, int64_t max_blocks, int3
     if (n_q > 0) off += align_up(attn_decode_partial_bytes());
     if (mode == QSA_MODE_PREFILL && max_blocks > 0 && n_q > 0) {
         L.pf_split = prefill_splits(n_q, max_blocks);
-        const size_t segs = (size_t)n_q * 2 * L.pf_split;
+        const size_t segs = (size_t)n_q * prefill_segments(L.pf_split);
         L.pf_cand = off;
         off += align_up(segs * prefill_seg_cap() * 8);
         L.pf_cnt = off;

@@ -71,7 +71,6 @@ k_cp_merge(const unsigned long long* __restrict__ keys_all, const int32_t* __res
 {
     __shared__ FinishSmem S;
     __shared__ int s_off[9];
-    __shared__ int s_nloc;
     const int tid = threadIdx.x;
     const int i = blockIdx.x;
     if (tid == 0) {
@@ -81,7 +80,6 @@ k_cp_merge(const unsigned long long* __restrict__ keys_all, const int32_t* __res
             s_off[r + 1] = s_off[r] + (c < 0 ? 0 : c > kSelCap ? kSelCap : c);
         }
         S.n_list = 0;
-        s_nloc = 0;
     }
     for (int k = tid; k < kSelCap; k += 256) S.list[k] = INT_MAX;
     __syncthreads();

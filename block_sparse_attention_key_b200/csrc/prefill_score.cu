@@ -29,7 +29,9 @@
 // histograms each row's scores (1/16-octave bins of the order-preserving key).
 // The main launch starts each row's admission threshold at the lower edge of the
 // bin holding its 64th-best sampled score (about 1,000 blocks of the row expected
-// above it) and then raises it as admitted scores fill a histogram: once `need`
+// above it; it lies above the row's 512th-best block only when at least 64 samples
+// fall among the 512 best blocks, a binomial with mean 32: probability about 4e-7)
+// and then raises it as admitted scores fill a histogram: once `need`
 // admitted blocks of a thread lie at or above a bin edge, no later block below it
 // can reach the top 512, and (blocks arrive in increasing index order) a later
 // block equal to it loses every tie, so the thread's own cut is strict.  Thresholds
@@ -758,6 +760,7 @@ int prefill_splits(int32_t n_q, int64_t max_blocks)
 }
 
 int prefill_seg_cap() { return 2048; }
+int prefill_segments(int n_split) { return 2 * n_split; }
 int prefill_shist_words(int n_split) { return 2 * n_split * kShistWords; }
 
 size_t prefill_smem_bytes() { return sizeof(K3Smem) + 1024; }

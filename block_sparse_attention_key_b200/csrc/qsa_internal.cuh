@@ -170,6 +170,7 @@ cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, i
 // streaming admission, exact finishing select, fallback for unsettled rows.
 int prefill_splits(int32_t n_q, int64_t max_blocks);
 int prefill_seg_cap();
+int prefill_segments(int n_split);  // admission segments per query row
 int prefill_shist_words(int n_split);
 bool prefill_sampled(const qsa_dims& d, int64_t max_blocks);
 cudaError_t launch_prefill_select(const qsa_dims& d, const void* q_idx, const float* w, const void* pooled,
