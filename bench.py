@@ -453,7 +453,7 @@ class Bench:
         res["attn_sets_per_graph"] = sets
         ach = (nbytes / sets) / (attn_ms / 1e3) / 1e9
         res["roofline_attention"] = {
-            "kernel": "k_attn_decode" if self.mode == qsa.QSA_MODE_DECODE else "k_sparse_attn", "bound": "hbm",
+            "kernel": "k_sparse_attn", "bound": "hbm",
             "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s", "frac": round(ach / hbm_peak, 4),
             "peak_source": f"{peak_kind} hbm_gbs (burst copy)", "algorithmic_bytes_per_launch": int(nbytes / sets)}
         if self.mode == qsa.QSA_MODE_PREFILL:

@@ -104,7 +104,7 @@ WsLayout plan_workspace(const qsa_dims& d, int32_t n_q, int64_t max_blocks, int3
     off += align_up((size_t)n_q * kSelCap * 4 + (size_t)n_q * 4);
     // decode attention partials, for a merge of split CTAs through global memory
     L.partial = off;
-    if (n_q > 0) off += align_up(attn_decode_partial_bytes());
+    if (n_q > 0) off += align_up(attn_partial_bytes());
     if (mode == QSA_MODE_PREFILL && max_blocks > 0 && n_q > 0) {
         L.pf_split = prefill_splits(n_q, max_blocks);
         const size_t segs = (size_t)n_q * prefill_segments(L.pf_split);
@@ -128,10 +128,8 @@ WsLayout plan_workspace(const qsa_dims& d, int32_t n_q, int64_t max_blocks, int3
     return L;
 }
 
-// Gathered attention for one call.  Calls with many (query, KV head) pairs, dense
-// caches and one query per selection (prefill chunks, large decode batches) run
-// k_sparse_attn, one CTA per pair at two CTAs per SM; everything else (few pairs:
-// splits over the block list; draft-query groups; paged caches) runs k_attn_decode.
+// Gathered attention for one call (k_sparse_attn): few (query group, KV head) pairs
+// split their block lists over the SMs, many pairs run one CTA per pair.
 static cudaError_t run_attention(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,
                                  const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,
                                  const int32_t* sel_cnt, const int32_t* page_table, int32_t page_tokens,
@@ -139,13 +137,9 @@ static cudaError_t run_attention(const qsa_dims& d, const void* q, const void* k
                                  char* ws, cudaStream_t st, bool pdl, bool counters_zeroed)
 {
     const int64_t n_groups = n_q / group_q;
-    const int64_t pairs = n_groups * d.n_kv_heads;
     float* partial = (float*)(ws + L.partial);
     unsigned* counters = (unsigned*)(ws + L.attn_cnt);
-    if (!page_table && group_q == 1 && pairs >= 2 * 148)
-        return launch_attention(d, q, k_cache, v_cache, q_seq, q_pos, sel_idx, sel_cnt, n_q, out, 1, partial,
-                                counters, (unsigned*)ws, st, pdl);
-    return launch_attn_decode(d, q, k_cache, v_cache, q_seq, q_pos, sel_idx, sel_cnt, page_table, page_tokens,
+    return launch_sparse_attn(d, q, k_cache, v_cache, q_seq, q_pos, sel_idx, sel_cnt, page_table, page_tokens,
                               n_pages, n_groups, group_q, out, partial, counters, (unsigned*)ws, st, pdl, true,
                               counters_zeroed);
 }
@@ -545,7 +539,7 @@ int qsa_cp_attn_partial(const qsa_dims* shard, const void* q, const void* k_shar
     unsigned* quiet = (unsigned*)ws + 1;
     cudaError_t e = launch_cp_local_pos(q_pos, n_q, blk_lo * shard->block_size, shard->kv_capacity, pos_loc, st);
     if (e == cudaSuccess)
-        e = launch_attn_decode(*shard, q, k_shard, v_shard, q_seq, pos_loc, sel_local, cnt_local, nullptr, 0, 0, n_q,
+        e = launch_sparse_attn(*shard, q, k_shard, v_shard, q_seq, pos_loc, sel_local, cnt_local, nullptr, 0, 0, n_q,
                                1, nullptr, (float*)(ws + L.partial), (unsigned*)(ws + L.attn_cnt), quiet, st, false,
                                true, true, part);
     return cuda_status(e);

@@ -85,9 +85,9 @@ extern "C" int qsa_sparse_attn_noalloc(const qsa_dims* dims, const void* q, cons
         return QSA_ERR_INVALID_ARG;
 
     const int64_t pairs = (int64_t)n_q * dims->n_kv_heads;
-    const int n_split = attn_decode_split_bound(pairs);
+    const int n_split = attn_split_bound(pairs);
     const size_t counter_bytes = ((size_t)pairs * 4 + kCounterAlign - 1) / kCounterAlign * kCounterAlign;
-    const size_t partial_bytes = n_split > 1 ? attn_decode_partial_bytes() : 0;
+    const size_t partial_bytes = n_split > 1 ? attn_partial_bytes() : 0;
     if (counter_bytes + partial_bytes > kScratchBytes) return QSA_ERR_WORKSPACE_TOO_SMALL;
 
     cudaStream_t st = (cudaStream_t)stream;
@@ -98,7 +98,7 @@ extern "C" int qsa_sparse_attn_noalloc(const qsa_dims* dims, const void* q, cons
     if (n_split > 1 && cudaMemsetAsync(counters, 0, (size_t)pairs * 4, st) != cudaSuccess) return QSA_ERR_CUDA;
     // no status word in this variant: out-of-range indices are still skipped, just not
     // reported; split partials always meet through the scratch array
-    const cudaError_t e = launch_attn_decode(*dims, q, k_cache, v_cache, q_seq, q_pos, sel_idx, sel_cnt, nullptr, 0,
+    const cudaError_t e = launch_sparse_attn(*dims, q, k_cache, v_cache, q_seq, q_pos, sel_idx, sel_cnt, nullptr, 0,
                                              0, n_q, 1, out, partial, counters, nullptr, st, false, false, true);
     return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
 }

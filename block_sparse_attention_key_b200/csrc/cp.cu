@@ -101,7 +101,7 @@ k_cp_merge(const unsigned long long* __restrict__ keys_all, const int32_t* __res
     if (want > 0) {
         const Cut cut = nc <= top_k ? Cut{0u, 0, true} : resolve_cut_regs(S, cr, nc, top_k, true, 0u);
         // keys equal at the cut come from distinct blocks: the lowest blocks win
-        take_by_cut(S, cr, nc, cut);
+        take_by_cut_exact(S, cr, nc, cut);
     }
     __syncthreads();
     sort_list_512(S);

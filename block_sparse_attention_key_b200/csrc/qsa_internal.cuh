@@ -179,13 +179,14 @@ cudaError_t launch_prefill_select(const qsa_dims& d, const void* q_idx, const fl
                                   uint32_t* shist, int32_t* worklist, float* scratch, int n_fallback_ctas,
                                   int32_t* sel_idx, int32_t* sel_cnt, unsigned* status, cudaStream_t st);
 
-// Decode-shaped gathered attention (attn_decode.cu): groups of `group_q` queries
-// sharing one selection row, optional paged K/V.  Splits of a (group, KV head) merge
-// in a thread-block cluster when allow_cluster and the device can hold every
-// cluster at once, else through `partial` / `counters` (counters zeroed by the caller).
-int attn_decode_split_bound(int64_t pairs);
-size_t attn_decode_partial_bytes();  // bytes of `partial` any launch needs
-cudaError_t launch_attn_decode(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,
+// Gathered attention (attn.cu): groups of `group_q` queries sharing one selection
+// row, optional paged K/V.  Few (group, KV head) pairs split their block lists; the
+// splits merge in a thread-block cluster when allow_cluster and the device can hold
+// every cluster at once, else through `partial` / `counters` (counters zeroed by the
+// caller).  Many pairs run one CTA per pair, two CTAs per SM.
+int attn_split_bound(int64_t pairs);
+size_t attn_partial_bytes();  // bytes of `partial` any launch needs
+cudaError_t launch_sparse_attn(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,
                                const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,
                                const int32_t* sel_cnt, const int32_t* page_table, int page_tokens, int64_t n_pages,
                                int64_t n_groups, int group_q, void* out, float* partial, unsigned* counters,
@@ -202,11 +203,5 @@ cudaError_t launch_cp_merge(const unsigned long long* keys_all, const int32_t* c
                             int top_k, int64_t blk_lo, int64_t n_local, int32_t* sel_local, int32_t* cnt_local,
                             int32_t* sel_global, int32_t* cnt_global, cudaStream_t st);
 cudaError_t launch_cp_combine(const float* parts, int n_ranks, int64_t rows, void* out, cudaStream_t st);
-
-cudaError_t launch_attention(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,
-                             const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,
-                             const int32_t* sel_cnt, int32_t n_q, void* out, int n_split, float* partial,
-                             unsigned* counters, unsigned* status, cudaStream_t st, bool pdl = false,
-                             bool cluster_merge = true);
 
 }  // namespace qsa

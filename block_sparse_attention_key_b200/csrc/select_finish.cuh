@@ -277,6 +277,42 @@ __device__ __forceinline__ bool take_by_cut(FinishSmem& S, const unsigned long l
     return true;
 }
 
+// take_by_cut for any number of keys tied at the cut: when too many tie to rank them
+// pairwise, the tied candidates' blocks (distinct) are cut by the same radix select
+// on ~block, so the `need` lowest blocks are taken.
+__device__ inline void take_by_cut_exact(FinishSmem& S, const unsigned long long (&cr)[kPerThreadCand], int nc,
+                                         const Cut& c)
+{
+    if (take_by_cut(S, cr, nc, c)) return;
+    const int tid = threadIdx.x;
+    unsigned long long tied[kPerThreadCand];
+#pragma unroll
+    for (int k = 0; k < kPerThreadCand; ++k)
+        tied[k] = (tid + 256 * k < nc && (unsigned)(cr[k] >> 32) == c.key)
+                      ? (unsigned long long)(~(uint32_t)cr[k]) << 32
+                      : 0ull;
+    const Cut cb = resolve_cut_regs(S, tied, nc, c.need, true, 0u);  // ~block values are distinct: cb.whole
+    unsigned take_mask = 0;
+#pragma unroll
+    for (int k = 0; k < kPerThreadCand; ++k) {
+        if (tid + 256 * k >= nc) continue;
+        const unsigned key = (unsigned)(cr[k] >> 32);
+        const bool take = key > c.key || (key == c.key && ~(uint32_t)cr[k] >= cb.key);
+        take_mask |= (take ? 1u : 0u) << k;
+    }
+    unsigned total;
+    int slot = S.n_list + (int)block_excl_scan_256((unsigned)__popc(take_mask), S.warp, &total);
+#pragma unroll
+    for (int k = 0; k < kPerThreadCand; ++k)
+        if (take_mask >> k & 1u) {
+            if (slot < kSelCap) S.list[slot] = (int)(unsigned)cr[k];
+            ++slot;
+        }
+    __syncthreads();
+    if (tid == 0) S.n_list += (int)total;
+    __syncthreads();
+}
+
 // Ordered selection of the top `need` keys of a score row in global memory
 // (keys whose top 12 bits exceed `p12` are all taken; among those equal to it the
 // top `need12`), written to S.list in ascending block order.  With `from_digit1`

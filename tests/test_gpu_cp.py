@@ -96,6 +96,57 @@ def test_cp_shards_reproduce_the_layer(R, bs):
     gu.compare_outputs(gu.bf16_to_f64(out), want)
 
 
+def test_cp_merge_breaks_score_ties_by_block():
+    """Every score equal (zero indexer queries): each of 4 shards keeps 512 tied keys,
+    the merge cuts 2,048 tied keys and must keep the 512 lowest blocks."""
+    import block_sparse_attention_key_b200 as qsa
+    import qsa_synth as syn
+    from block_sparse_attention_key_b200 import cp
+    wl, dw, T = _setup()
+    n, R, bs = T["n_q"], 4, wl.block_size
+    q_idx0 = torch.zeros_like(T["q_idx"])
+    shards = [cp.shard_range(wl.kv_capacity // bs, R, r) for r in range(R)]
+    keys_all = torch.zeros((R, n, qsa.QSA_SEL_CAP), dtype=torch.int64, device="cuda")
+    cnt_all = torch.zeros((R, n), dtype=torch.int32, device="cuda")
+    state = []
+    for r, (lo, nb) in enumerate(shards):
+        sd = qsa.make_dims(wl.batch, wl.n_q_heads, wl.n_kv_heads, nb * bs, block_size=bs, top_k=wl.top_k)
+        ks, vs, ps = _shard_tensors(wl, dw, lo, nb)
+        ws = gu.new_workspace(qsa.qsa_cp_workspace_bytes(sd, n))
+        qsa.qsa_cp_select_keys(sd, q_idx0, T["w"], ps, T["q_seq"], T["q_pos"], n, lo, keys_all[r], cnt_all[r], ws)
+        state.append((sd, ks, vs, ws, lo))
+    parts = torch.zeros((R, n, wl.n_q_heads, qsa.CP_PART_ROW), dtype=torch.float32, device="cuda")
+    for r, (sd, ks, vs, ws, lo) in enumerate(state):
+        sel_l = torch.empty((n, qsa.QSA_SEL_CAP), dtype=torch.int32, device="cuda")
+        cnt_l = torch.empty((n,), dtype=torch.int32, device="cuda")
+        sel_g = torch.empty_like(sel_l)
+        cnt_g = torch.empty_like(cnt_l)
+        qsa.qsa_cp_merge_keys(sd, R, keys_all, cnt_all, n, lo, sel_l, cnt_l, sel_g, cnt_g)
+        qsa.qsa_cp_attn_partial(sd, T["q"], ks, vs, T["q_seq"], T["q_pos"], n, lo, sel_l, cnt_l, parts[r], ws)
+        sg, cg = sel_g.cpu().numpy(), cnt_g.cpu().numpy()
+        for i in range(n):
+            n_c = (wl.steps[0].q_pos[i] + 1) // bs
+            np.testing.assert_array_equal(sg[i, : cg[i]], np.arange(min(n_c, wl.top_k)), err_msg=f"query {i}")
+    out = torch.empty((n, wl.n_q_heads, 128), dtype=torch.bfloat16, device="cuda")
+    qsa.qsa_cp_combine(gu.dims_of(wl), R, parts, n, out)
+    torch.cuda.synchronize()
+    # the oracle with the same (zero) indexer queries
+    wo = O.WorkloadOracle(wl)
+    st = wl.steps[0]
+    zero_bits = gu.to_bits(torch.zeros((wl.n_idx_heads, wl.idx_dim), dtype=torch.bfloat16))
+    want = np.zeros((n, wl.n_q_heads, 128))
+    for i in range(n):
+        s_, t, qid = st.q_seq[i], st.q_pos[i], st.query_ids[i]
+        pooled = wo.pooled(s_, (t + 1) // bs)
+        w_ = syn.gen_w(wl.seed, [qid], wl.n_idx_heads)[0]
+        q_ = syn.gen_q(wl.seed, [qid], wl.n_q_heads, wl.head_dim)[0]
+        fetch = lambda toks, s_=s_: (syn.gen_kv_rows(wl.seed, "k", s_, toks, wl.n_kv_heads, wl.head_dim),
+                                     syn.gen_kv_rows(wl.seed, "v", s_, toks, wl.n_kv_heads, wl.head_dim))
+        sel, want[i] = O.query_forward(pooled, zero_bits, w_, t, q_, fetch, wl.top_k, bs)
+        np.testing.assert_array_equal(sel, np.arange(min((t + 1) // bs, wl.top_k)))
+    gu.compare_outputs(gu.bf16_to_f64(out), want)
+
+
 def test_cp_decode_over_a_process_group():
     """The orchestrating module end to end with real NCCL collectives (one rank)."""
     import os

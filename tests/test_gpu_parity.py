@@ -400,6 +400,17 @@ def test_forward_prefill_interleaved_sequences():
     _forward_vs_oracle(wl)
 
 
+def test_forward_prefill_three_sequences_at_long_capacity():
+    """A prefill call over three sequences of a 393,216-token cache: rows whose
+    blocks all lie in the first 131,072 tokens, rows straddling token 131,072
+    (partial block on either side), rows at 300,000; every row against the oracle."""
+    q_seq = [0] * 60 + [1] * 40 + [2] * 60
+    q_pos = list(range(131040, 131100)) + list(range(300000, 300040)) + list(range(100, 160))
+    wl = W.Workload("pf_passes", 89, "prefill", 3, 16, 2, 3 * 131072,
+                    [W.Step([131040, 300000, 100], [131100, 300040, 160], q_seq, q_pos, list(range(len(q_pos))))])
+    _forward_vs_oracle(wl)
+
+
 @pytest.mark.parametrize("cap", [8192, 65536, 131072])
 def test_forward_decode_ties_take_lowest_blocks(cap):
     """Decode rows whose scores tie massively at the cut (the select inside the
