@@ -15,15 +15,19 @@
 // scores only in its own sequence's pass.
 //
 // CTA = 10 warps, one CTA per SM (512 TMEM columns):
-//   warp 0      TMA producer: the 4 query tiles once, then 64-block pooled tiles
-//               (8 KiB, 128-byte swizzle) into an 8-deep ring;
+//   warp 0      TMA producer: the 4 query tiles once, then 128-block pooled tiles
+//               (16 KiB, 128-byte swizzle) into a 4-deep ring;
 //   warp 1      TMEM allocator and MMA issuer: per pooled tile, 4 heads x 4 K-steps of
-//               tcgen05.mma (M=128, N=64, K=16, bf16 -> f32) into accumulator stage
-//               (tile & 1), 4 heads x 64 columns each;
-//   warps 2..9  epilogue, two warpgroups: warpgroup g takes the tiles with
-//               (tile & 1) == g, so while one loads TMEM the other computes; each
-//               thread owns one query row (its TMEM lane): tcgen05.ld, ReLU, weights
-//               (packed f32x2 FMAs), head sum, causal cut, streaming admission.
+//               tcgen05.mma (M=128, N=128, K=16, bf16 -> f32): heads 0 and 1 into
+//               accumulator buffer A (TMEM columns 0..255), heads 2 and 3 into buffer
+//               B (256..511), so the next tile's first head pair is computed while the
+//               epilogue reads this tile's second (N=128 runs the tensor pipe at its
+//               full rate, N=64 at two thirds, and halves the MMAs issued per block);
+//   warps 2..9  epilogue, two warpgroups: warpgroup g takes columns 64g..64g+63 of
+//               every tile; each thread owns one query row (its TMEM lane): tcgen05.ld
+//               of buffer A, the partial sum w0 ReLU(s0) + w1 ReLU(s1) (packed f32x2
+//               FMAs), buffer A released, then buffer B completes the chain with heads
+//               2 and 3 and is released; causal cut, streaming admission.
 //
 // Two launches per chunk.  A sampling launch scores every 16th block and only
 // histograms each row's scores (1/16-octave bins of the order-preserving key).
@@ -58,8 +62,8 @@ using namespace sm100;
 namespace {
 
 constexpr int kM = 128;                 // query rows per CTA
-constexpr int kN = 64;                  // pooled blocks per tile
-constexpr int kNumB = 8;                // pooled-tile ring depth
+constexpr int kN = 128;                 // pooled blocks per tile
+constexpr int kNumB = 4;                // pooled-tile ring depth
 constexpr int kEpiWarps = 8;
 constexpr int kK3Threads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
@@ -75,7 +79,7 @@ constexpr uint32_t kNoWindow = 0xFFFFFFFFu;  // window base of a sampler that sa
 
 struct __align__(1024) K3Smem {
     __nv_bfloat16 a[kIdxHeads][kM * kIdxDim];   // 4 x 16 KiB
-    __nv_bfloat16 b[kNumB][kN * kIdxDim];       // 8 x 8 KiB
+    __nv_bfloat16 b[kNumB][kN * kIdxDim];       // 4 x 16 KiB
     uint32_t hist[2][kHistBins][kM];            // 64 KiB, counter-major per warpgroup
     float w[kM][kIdxHeads];
     int n_c[kM];
@@ -84,7 +88,7 @@ struct __align__(1024) K3Smem {
     int pass_ncmax[kM];  // longest row of each pass
     int n_pass;
     uint64_t full[kNumB], empty[kNumB];
-    uint64_t tmem_full[2], tmem_empty[2];
+    uint64_t tmem_full[2], tmem_empty[2];       // accumulator buffers A (heads 0, 1) and B (heads 2, 3)
     uint64_t a_full, mma_done;
     uint32_t tmem_base;
     int error;
@@ -158,20 +162,32 @@ __device__ __forceinline__ float max3(float a, float b, float c)
     return d;
 }
 
-// 32 scores of one row: sum_h w_h * ReLU(a_h[c]), the same FMA chain as the decode
-// scorer (w0*r0, then + w1*r1, + w2*r2, + w3*r3), two columns per packed f32x2 FMA.
-__device__ __forceinline__ void row_scores32(const float (&a)[kIdxHeads][32], unsigned long long w0,
-                                             unsigned long long w1, unsigned long long w2, unsigned long long w3,
-                                             float (&sc)[32])
+// 32 consecutive TMEM columns of this thread's lane (two 16-column loads; the caller waits).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    float lo[16], hi[16];
+    tmem_ld16(taddr, lo);
+    tmem_ld16(taddr + 16, hi);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+        v[c] = lo[c];
+        v[16 + c] = hi[c];
+    }
+}
+
+// Two heads of 32 columns of one row folded into the score chain (the same FMA
+// order as the decode scorer: w0*r0, then + w1*r1, + w2*r2, + w3*r3), two columns
+// per packed f32x2 FMA: acc[c] = wb * ReLU(b[c]) + (wa * ReLU(a[c]) + (cont ? acc[c] : 0)).
+__device__ __forceinline__ void pair_scores32(const float (&a)[32], const float (&b)[32], unsigned long long wa,
+                                              unsigned long long wb, float (&acc)[32], bool cont)
 {
 #pragma unroll
     for (int c = 0; c < 32; c += 2) {
-        unsigned long long s = fma2(w0, pack2(fmaxf(a[0][c], 0.f), fmaxf(a[0][c + 1], 0.f)), 0ull);
-        s = fma2(w1, pack2(fmaxf(a[1][c], 0.f), fmaxf(a[1][c + 1], 0.f)), s);
-        s = fma2(w2, pack2(fmaxf(a[2][c], 0.f), fmaxf(a[2][c + 1], 0.f)), s);
-        s = fma2(w3, pack2(fmaxf(a[3][c], 0.f), fmaxf(a[3][c + 1], 0.f)), s);
-        sc[c] = __uint_as_float((unsigned)s);
-        sc[c + 1] = __uint_as_float((unsigned)(s >> 32));
+        unsigned long long s = cont ? pack2(acc[c], acc[c + 1]) : 0ull;
+        s = fma2(wa, pack2(fmaxf(a[c], 0.f), fmaxf(a[c + 1], 0.f)), s);
+        s = fma2(wb, pack2(fmaxf(b[c], 0.f), fmaxf(b[c + 1], 0.f)), s);
+        acc[c] = __uint_as_float((unsigned)s);
+        acc[c + 1] = __uint_as_float((unsigned)(s >> 32));
     }
 }
 
@@ -201,7 +217,7 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.tmem_full[i], 1);
-            mbar_init(&S.tmem_empty[i], kEpiWarps / 2);
+            mbar_init(&S.tmem_empty[i], kEpiWarps);  // every epilogue warp reads both buffers
         }
         mbar_init(&S.a_full, 1);
         mbar_init(&S.mma_done, 1);
@@ -321,20 +337,28 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
             for (int h = 0; h < kIdxHeads; ++h) adesc[h] = smem_desc_sw128(smem_u32(S.a[h]));
             if (wait_phase(&S.a_full, 0, err, status)) {
                 for (int j = 0; j < n_stages; ++j) {  // every pass's stages in order
-                    const int slot = j % kNumB, ts = j & 1;
+                    const int slot = j % kNumB;
                     if (!wait_phase(&S.full[slot], (j / kNumB) & 1, err, status)) break;
-                    if (j >= 2 && !wait_phase(&S.tmem_empty[ts], ((j >> 1) - 1) & 1, err, status)) break;
-                    tc_fence_after();
                     const uint64_t bdesc = smem_desc_sw128(smem_u32(S.b[slot]));
-                    // K-step outer, head inner: consecutive MMAs write different
-                    // accumulators, so they overlap instead of waiting on each other
+                    bool ok = true;
+                    for (int pr = 0; pr < 2 && ok; ++pr) {
+                        // head pair pr into buffer pr, once the epilogue has read the previous tile's
+                        if (j >= 1 && !wait_phase(&S.tmem_empty[pr], (j - 1) & 1, err, status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        // K-step outer, head inner: consecutive MMAs write different accumulators
 #pragma unroll
-                    for (int k = 0; k < kIdxDim / 16; ++k)
+                        for (int k = 0; k < kIdxDim / 16; ++k)
 #pragma unroll
-                        for (int h = 0; h < kIdxHeads; ++h)
-                            mma_bf16_ss(tmem + ts * 256 + h * kN, adesc[h] + 2 * k, bdesc + 2 * k, idesc, k > 0);
+                            for (int hh = 0; hh < 2; ++hh)
+                                mma_bf16_ss(tmem + pr * 256 + hh * kN, adesc[2 * pr + hh] + 2 * k, bdesc + 2 * k, idesc,
+                                            k > 0);
+                        mma_commit(&S.tmem_full[pr]);
+                    }
+                    if (!ok) break;
                     mma_commit(&S.empty[slot]);
-                    mma_commit(&S.tmem_full[ts]);
                 }
             }
             // every MMA issued must finish before TMEM is released
@@ -358,7 +382,7 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
         uint32_t* hist = &S.hist[wg][0][0] + row;  // counter k at hist[k * kM]
         int wb = -1;                               // histogram window base (absolute bin)
         unsigned wcount = 0;                       // keys counted in the window
-        const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + wg * 256;
+        const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16);  // this warp's 32 TMEM lanes
 
         // ---- main-pass state ----
         unsigned long long* seg = cand + ((row_g * n_split + split) * 2 + wg) * (int64_t)seg_cap;
@@ -401,45 +425,62 @@ k_prefill_scores_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_con
             const int nc = my_seq == S.pass_seq[p] ? nc_own : 0;
             const bool live = live_any && nc > 0;
             for (int jp = 0; jp < n_st; ++jp, ++J) {
-                if ((J & 1) != wg) continue;
-                const int j = jp;          // stage within the pass
-                const int k_own = J >> 1;  // this warpgroup's k-th tile
-                if (!wait_phase(&S.tmem_full[wg], k_own & 1, err, status)) {
+                const int j = jp;  // stage within the pass
+                // buffer A: heads 0 and 1 of this warpgroup's 64 columns -> partial sums
+                if (!wait_phase(&S.tmem_full[0], J & 1, err, status)) {
                     stop = true;
                     break;
                 }
                 tc_fence_after();
-                if (!kSample && (k_own & 7) == 7 && live) {
+                if (!kSample && (J & 7) == 7 && live) {
                     const unsigned g = __ldcg(theta_g + row_g);
                     if (g > theta_key) {
                         theta_key = g;
                         theta_f = key_to_float(theta_key);
                     }
                 }
+                float part0[32], part1[32];  // columns 0..31 and 32..63 of this warpgroup's share
+                {
+                    float a0[32], a1[32];
+                    tmem_ld32(tbase + 0 * kN + wg * 64, a0);
+                    tmem_ld32(tbase + 1 * kN + wg * 64, a1);
+                    tmem_ld_wait();
+                    pair_scores32(a0, a1, w0, w1, part0, false);
+                    tmem_ld32(tbase + 0 * kN + wg * 64 + 32, a0);
+                    tmem_ld32(tbase + 1 * kN + wg * 64 + 32, a1);
+                    tmem_ld_wait();
+                    pair_scores32(a0, a1, w0, w1, part1, false);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.tmem_empty[0]);
+                // buffer B: heads 2 and 3 complete the chain w0 r0 + w1 r1 + w2 r2 + w3 r3
+                if (!wait_phase(&S.tmem_full[1], J & 1, err, status)) {
+                    stop = true;
+                    break;
+                }
+                tc_fence_after();
+                {
+                    float a2[32], a3[32];
+                    tmem_ld32(tbase + 2 * kN + wg * 64, a2);
+                    tmem_ld32(tbase + 3 * kN + wg * 64, a3);
+                    tmem_ld_wait();
+                    pair_scores32(a2, a3, w2, w3, part0, true);
+                    tmem_ld32(tbase + 2 * kN + wg * 64 + 32, a2);
+                    tmem_ld32(tbase + 3 * kN + wg * 64 + 32, a3);
+                    tmem_ld_wait();
+                    pair_scores32(a2, a3, w2, w3, part1, true);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.tmem_empty[1]);
+                if (!live) continue;
 #pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
-                    float a[kIdxHeads][32];
-#pragma unroll
-                    for (int h = 0; h < kIdxHeads; ++h) {
-                        float lo[16], hi[16];
-                        tmem_ld16(tbase + h * kN + half * 32, lo);
-                        tmem_ld16(tbase + h * kN + half * 32 + 16, hi);
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            a[h][c] = lo[c];
-                            a[h][16 + c] = hi[c];
-                        }
-                    }
-                    tmem_ld_wait();
-                    if (half == 1) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&S.tmem_empty[wg]);
-                    }
-                    if (!live) continue;
                     float sc[32];
-                    row_scores32(a, w0, w1, w2, w3, sc);
-                    const int b_base = blk0 + j * kN + half * 32;
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) sc[c] = half ? part1[c] : part0[c];
+                    const int b_base = blk0 + j * kN + wg * 64 + half * 32;
                     if (b_base + 32 > nc) {
 #pragma unroll
                         for (int c = 0; c < 32; ++c)
@@ -607,7 +648,7 @@ __device__ __forceinline__ void gather_segments(const unsigned long long* __rest
 // or above the row's final threshold), or every block when n_c <= 512.  Rows whose
 // segments overflowed, or whose survivors do not fit the shared-memory finisher,
 // go to the worklist of k_prefill_fallback.
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 3)  // three rows per SM
 k_prefill_finish(const int32_t* __restrict__ q_seq, const int32_t* __restrict__ q_pos, int32_t n_q, int32_t batch,
                  int64_t kv_capacity, int64_t max_blocks, int bs, int top_k, int n_split, int seg_cap,
                  const unsigned long long* __restrict__ cand, const unsigned* __restrict__ cand_cnt,
