@@ -10,7 +10,10 @@ is the whole layer through the C ABI (qsa_forward): pool the appended token's
 block, score every complete causal block, select the top 512, gathered attention.
 Inputs sit in HBM when the timed region starts; L2 is flushed (a 512 MiB write,
 then a 512 MiB read) before every timed step, outside the timed events.  Rank 0 prints
-one JSON line.  `--impl reference` times the CPU oracle on the same workload.
+one JSON line.  After the headline (unless --no-workload-map) the line also carries
+every other configuration (`workloads`) and two serving shapes on the headline's
+geometry (`serving_modes`: 4 draft queries per sequence sharing one selection, and
+K/V in 256-token pages).  `--impl reference` times the CPU oracle on the same workload.
 """
 
 import argparse
@@ -527,6 +530,75 @@ class Bench:
                           "output, stream sync"}
 
 
+def serving_modes(env, args):
+    """Serving shapes on the headline's geometry (16 sequences at 64K context, 32 / 4
+    heads), each timed like the headline (CUDA-graph replays of qsa_forward, L2
+    flushed before each): 4 draft queries per sequence sharing one selection
+    (multi-token prediction), and the K/V caches held in 256-token pages at a random
+    page order."""
+    torch, qsa, sdev = env.torch, env.qsa, env.sdev
+    from qsa_synth import workloads as W
+    out = {}
+    for name, k, page_tokens in (("mtp4_decode_64k_b16", 4, 0), ("paged256_decode_64k_b16", 1, 256)):
+        cap, batch = 65536, 16
+        t0 = cap - k
+        q_seq = [s for s in range(batch) for _ in range(k)]
+        q_pos = [t0 + j for _ in range(batch) for j in range(k)]
+        wl = W.Workload(name, 201 + k, "decode", batch, 32, 4, cap,
+                        [W.Step([t0] * batch, [cap] * batch, q_seq, q_pos, list(range(len(q_pos))))])
+        dw = sdev.DeviceWorkload(wl)
+        zeros = torch.zeros(batch, dtype=torch.int32, device="cuda")
+        dims = qsa.make_dims(batch, 32, 4, cap, block_size=wl.block_size, top_k=wl.top_k)
+        qsa.qsa_pool_block_keys(dims, dw.idx_k, dw.pooled, zeros,
+                                torch.tensor([t0] * batch, dtype=torch.int32, device="cuda"), t0)
+        T = dw.step_tensors(0)
+        n = T["n_q"]
+        kc, vc, table, n_pages = dw.k_cache, dw.v_cache, None, 0
+        if page_tokens:
+            B, H, Tt, D = dw.k_cache.shape
+            per_seq = Tt // page_tokens
+            n_pages = B * per_seq
+            perm = torch.tensor(np.random.default_rng(7).permutation(n_pages).reshape(B, per_seq).astype(np.int32),
+                                device="cuda")
+            kc = torch.empty((n_pages, H, page_tokens, D), dtype=torch.bfloat16, device="cuda")
+            vc = torch.empty_like(kc)
+            kc[perm.long().reshape(-1)] = dw.k_cache.view(B, H, per_seq, page_tokens, D).permute(0, 2, 1, 3, 4).reshape(-1, H, page_tokens, D)
+            vc[perm.long().reshape(-1)] = dw.v_cache.view(B, H, per_seq, page_tokens, D).permute(0, 2, 1, 3, 4).reshape(-1, H, page_tokens, D)
+            table = perm
+            del dw.k_cache, dw.v_cache
+            torch.cuda.empty_cache()
+        ws = torch.empty(qsa.qsa_workspace_bytes(dims, n, T["max_blocks"], qsa.QSA_MODE_DECODE), dtype=torch.uint8,
+                         device="cuda")
+        qsa.qsa_workspace_init(ws)
+        o = torch.empty((n, 32, 128), dtype=torch.bfloat16, device="cuda")
+        sel = torch.empty((n // k, qsa.QSA_SEL_CAP), dtype=torch.int32, device="cuda")
+        cnt = torch.empty((n // k,), dtype=torch.int32, device="cuda")
+        q_idx, w = T["q_idx"][::k].contiguous(), T["w"][::k].contiguous()
+
+        def fwd():
+            qsa.qsa_forward(dims, q=T["q"], k_cache=kc, v_cache=vc, idx_k=dw.idx_k, pooled=dw.pooled, q_idx=q_idx,
+                            w=w, len_before=T["len_before"], len_after=T["len_after"], q_seq=T["q_seq"],
+                            q_pos=T["q_pos"], n_q=n, max_new_tokens=T["max_new_tokens"], max_blocks=T["max_blocks"],
+                            mode=qsa.QSA_MODE_DECODE, out=o, workspace=ws, sel_idx=sel, sel_cnt=cnt, group_q=k,
+                            page_table=table, page_tokens=page_tokens, n_pages=n_pages)
+        for _ in range(max(args.warmup, 3)):
+            fwd()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fwd()
+        g.replay()
+        torch.cuda.synchronize()
+        ms = env.max_ms(float(np.mean(env.timed(g.replay, args.steps))))
+        del g
+        out[name] = {"tokens_per_s": job_tokens_per_s(1, n, ms), "ms_per_unit": ms, "queries_per_unit": n,
+                     "selections_per_unit": n // k, "draft_queries_per_selection": k, "page_tokens": page_tokens,
+                     "device_status": qsa.qsa_read_device_status(ws)}
+        del dw, kc, vc, ws
+        torch.cuda.empty_cache()
+    return out
+
+
 ATTN_SETS = {"decode_8k_b1": 16, "decode_64k_b16": 8, "decode_1m_b4": 8}
 
 
@@ -593,6 +665,7 @@ def run_ours(args, wl):
             del Bo
             torch.cuda.empty_cache()
         line["workloads"] = wmap
+        line["serving_modes"] = serving_modes(env, args)
         line["workloads_note"] = ("each configuration measured alone on this GPU after the headline: CUDA-graph "
                                   "replays of its whole unit with L2 flushed before each; selection and attention "
                                   "timed through their standalone entry points")

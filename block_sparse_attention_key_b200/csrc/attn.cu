@@ -278,11 +278,14 @@ k_sparse_attn(const uint4* __restrict__ q, const uint16_t* __restrict__ k_cache,
 
     const int tlast = s_tlast;
     const int n_tiles = (n_blk + ipt - 1) / ipt;
+    // four threads per token row, each copying chunks q, q + 4, q + 8, q + 12 (16 B each):
+    // one row lookup per thread and tile, 64 contiguous bytes per row per copy instruction
+    constexpr int kRowsPerPass = kT / 4;
     auto load_tile = [&](int tile, int slot) {
+        const int q4 = tid & 3;
 #pragma unroll
-        for (int u = 0; u < (kTT * 16) / kT; ++u) {
-            const int idx = tid + u * kT;
-            const int row = idx >> 4, ch = idx & 15;
+        for (int u = 0; u < kTT / kRowsPerPass; ++u) {
+            const int row = (tid >> 2) + u * kRowsPerPass;
             const int it = tile * ipt + (row >> bs_log2);
             const int tin = row & (bs - 1);
             long long off = -1;
@@ -294,11 +297,15 @@ k_sparse_attn(const uint4* __restrict__ q, const uint16_t* __restrict__ k_cache,
                 if (off >= 0) tp = ip < 0 ? -1 : ip + tin;
             }
             const bool valid = off >= 0;
-            const long long e = valid ? off + (long long)tin * kHeadDim + ch * 8 : 0;
-            const uint32_t so = swz(row, ch) + slot * kStage;
-            cp_async16(sbase + SL.k + so, k_cache + e, valid ? 16 : 0);
-            cp_async16(sbase + SL.v + so, v_cache + e, valid ? 16 : 0);
-            if (ch == 0) s_tok[slot * kTT + row] = tp;
+            const long long e = valid ? off + (long long)tin * kHeadDim : 0;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int ch = q4 + 4 * k;
+                const uint32_t so = swz(row, ch) + slot * kStage;
+                cp_async16(sbase + SL.k + so, k_cache + e + (valid ? ch * 8 : 0), valid ? 16 : 0);
+                cp_async16(sbase + SL.v + so, v_cache + e + (valid ? ch * 8 : 0), valid ? 16 : 0);
+            }
+            if (q4 == 0) s_tok[slot * kTT + row] = tp;
         }
     };
 
