@@ -18,7 +18,7 @@ constexpr int kMaxBlockSize = 16;
 constexpr int kIdxHeads = 4;     // indexer heads
 constexpr int kIdxDim = 64;      // indexer head dim
 constexpr int kHeadDim = 128;    // main attention head dim
-constexpr int kMaxGroup = 16;    // query heads per KV head handled by one attention CTA
+constexpr int kMaxGroup = 32;    // query heads per KV head handled by one attention CTA
 
 // ---- top-k radix select: 32-bit orderable keys, digits of 12 + 12 + 8 bits ----
 constexpr int kBins1 = 4096;

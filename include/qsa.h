@@ -96,7 +96,7 @@ extern "C" {
 
 typedef struct qsa_dims {
     int32_t batch;        /* B, number of sequences (caches) */
-    int32_t n_q_heads;    /* main attention query heads (multiple of n_kv_heads, group <= 16) */
+    int32_t n_q_heads;    /* main attention query heads (multiple of n_kv_heads, group <= 32) */
     int32_t n_kv_heads;   /* main attention KV heads */
     int32_t head_dim;     /* must be 128 */
     int32_t n_idx_heads;  /* indexer heads, must be 4 */

@@ -176,7 +176,7 @@ def test_topk_partial_positions_use_complete_blocks_only():
 
 # ------------------------------------------------------------------ step 4: attention
 
-@pytest.mark.parametrize("hq,hkv", [(8, 1), (32, 4), (16, 16), (16, 1), (4, 2)])
+@pytest.mark.parametrize("hq,hkv", [(8, 1), (32, 4), (16, 16), (16, 1), (4, 2), (32, 1)])
 def test_sparse_attn_matches_oracle(hq, hkv):
     import block_sparse_attention_key_b200 as qsa
     from qsa_synth import device as sdev
@@ -211,6 +211,45 @@ def test_sparse_attn_matches_oracle(hq, hkv):
         toks = O.attended_tokens(sel[r, : cnt[r]], t)
         k = syn.gen_kv_rows(wl.seed, "k", s, toks, hkv, 128)
         v = syn.gen_kv_rows(wl.seed, "v", s, toks, hkv, 128)
+        want[r] = O.gqa_attention(qbits[r], k, v)
+    gu.compare_outputs(got, want)
+
+
+@pytest.mark.parametrize("hq,hkv", [(32, 1), (32, 2), (16, 8), (8, 1)])
+def test_sparse_attn_many_pairs_matches_oracle(hq, hkv):
+    """At least 148 (query, KV head) pairs: one CTA per pair, queries-fastest grid, for
+    every row count of the kernel (group sizes 32, 16, 2 and 8 query heads per KV
+    head); random selections and positions, partial blocks included."""
+    import block_sparse_attention_key_b200 as qsa
+    from qsa_synth import device as sdev
+    rng = np.random.default_rng(hq * 1000 + hkv)
+    cap, n = 4096, 160
+    positions = [int(x) for x in rng.integers(0, cap, n)]
+    seqs = [int(x) for x in rng.integers(0, 2, n)]
+    wl = small_workload(f"attn_pairs{hq}_{hkv}", 2, hq, hkv, cap,
+                        [W.Step([cap] * 2, [cap] * 2, seqs, positions, list(range(n)))])
+    dw = sdev.DeviceWorkload(wl)
+    T = dw.step_tensors(0)
+    sel = np.full((n, 512), -1, dtype=np.int32)
+    cnt = np.zeros(n, dtype=np.int32)
+    for r, t in enumerate(positions):
+        n_c = (t + 1) // 4
+        k = min(512, n_c)
+        sel[r, :k] = np.sort(rng.choice(n_c, size=k, replace=False)) if k else np.zeros(0, np.int64)
+        cnt[r] = k
+    dims = gu.dims_of(wl)
+    ws = gu.new_workspace(qsa.qsa_workspace_bytes(dims, n, 0, 0))
+    out = torch.empty((n, hq, 128), dtype=torch.bfloat16, device="cuda")
+    qsa.qsa_sparse_attn(dims, T["q"], dw.k_cache, dw.v_cache, T["q_seq"], T["q_pos"], torch.tensor(sel, device="cuda"),
+                        torch.tensor(cnt, device="cuda"), n, out, ws)
+    assert qsa.qsa_read_device_status(ws) == 0
+    got = gu.bf16_to_f64(out)
+    want = np.zeros_like(got)
+    qbits = gu.to_bits(T["q"])
+    for r, (s_, t) in enumerate(zip(seqs, positions)):
+        toks = O.attended_tokens(sel[r, : cnt[r]], t)
+        k = syn.gen_kv_rows(wl.seed, "k", s_, toks, hkv, 128)
+        v = syn.gen_kv_rows(wl.seed, "v", s_, toks, hkv, 128)
         want[r] = O.gqa_attention(qbits[r], k, v)
     gu.compare_outputs(got, want)
 
