@@ -10,4 +10,5 @@ from .qsa import (  # noqa: F401
     qsa_index_scores, qsa_topk_blocks, qsa_sparse_attn, qsa_forward, qsa_sparse_attn_noalloc,
     qsa_sparse_attn_ex, qsa_select_blocks, QSA_DEV_BAD_PAGE, QSA_SEL_CAP, CP_PART_ROW,
     qsa_cp_workspace_bytes, qsa_cp_select_keys, qsa_cp_merge_keys, qsa_cp_attn_partial, qsa_cp_combine,
+    qsa_attn_plan,
 )

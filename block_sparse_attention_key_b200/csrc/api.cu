@@ -364,6 +364,30 @@ int qsa_sparse_attn_ex(const qsa_dims* dims, const qsa_attn_args* a, void* works
                                      (char*)workspace, (cudaStream_t)stream, false, true));
 }
 
+int qsa_attn_plan(const qsa_dims* dims, int32_t n_q, int32_t group_q, qsa_attn_plan_info* info)
+{
+    int rc = check_dims(dims);
+    if (rc != QSA_OK) return rc;
+    if (!info) return QSA_ERR_INVALID_ARG;
+    if ((rc = check_rows(dims, n_q, 0)) != QSA_OK) return rc;
+    if ((rc = check_groups(dims, n_q, group_q < 1 ? 0 : group_q)) != QSA_OK) return rc;
+    *info = qsa_attn_plan_info{};
+    if (n_q == 0) return QSA_OK;
+    int n_split = 0, stages = 0, threads = 0, smem = 0, cluster = 0, rows = 0;
+    int64_t ctas = 0;
+    if (!describe_sparse_attn(*dims, n_q / group_q, group_q, true, &n_split, &stages, &threads, &smem, &ctas, &cluster,
+                              &rows))
+        return QSA_ERR_UNSUPPORTED;
+    info->n_split = n_split;
+    info->n_stages = stages;
+    info->threads = threads;
+    info->smem_bytes = smem;
+    info->ctas = ctas;
+    info->cluster_merge = cluster;
+    info->rows = rows;
+    return QSA_OK;
+}
+
 int qsa_select_blocks(const qsa_dims* dims, const void* q_idx, const float* w, const void* pooled,
                       const int32_t* q_seq, const int32_t* q_pos, int32_t n_q, int64_t max_blocks, int32_t mode,
                       int32_t* sel_idx, int32_t* sel_cnt, void* workspace, size_t ws_bytes, void* stream)

@@ -744,6 +744,33 @@ Plan plan(int dev, int64_t pairs, int rows, bool allow_cluster, int ipt)
 
 }  // namespace
 
+bool describe_sparse_attn(const qsa_dims& d, int64_t n_groups, int group_q, bool allow_cluster, int* n_split,
+                          int* stages, int* threads, int* smem, int64_t* ctas, int* cluster, int* rows)
+{
+    const int G = d.n_q_heads / d.n_kv_heads;
+    const int r = G * group_q;
+    if (r > 32 || n_groups <= 0) return false;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || !configure(dev, nt_for_rows(r))) {
+        // no device: the plan without the occupancy query of the cluster merge
+        cudaGetLastError();
+        dev = 0;
+        allow_cluster = false;
+    }
+    int bs_log2 = 0;
+    while ((1 << bs_log2) < d.block_size) ++bs_log2;
+    const int64_t pairs = n_groups * d.n_kv_heads;
+    const Plan p = plan(dev, pairs, r, allow_cluster, kTT >> bs_log2);
+    *n_split = p.n_split;
+    *stages = p.stages;
+    *threads = 128 * nwg_for(nt_for_rows(r));
+    *smem = p.smem;
+    *ctas = pairs * p.n_split;
+    *cluster = p.cluster ? 1 : 0;
+    *rows = r;
+    return true;
+}
+
 int attn_split_bound(int64_t pairs)
 {
     if (pairs <= 0 || pairs >= 148) return 1;

@@ -185,6 +185,9 @@ cudaError_t launch_prefill_select(const qsa_dims& d, const void* q_idx, const fl
 // every cluster at once, else through `partial` / `counters` (counters zeroed by the
 // caller).  Many pairs run one CTA per pair, two CTAs per SM.
 int attn_split_bound(int64_t pairs);
+// The launch shape of launch_sparse_attn for n_groups groups (host arithmetic only).
+bool describe_sparse_attn(const qsa_dims& d, int64_t n_groups, int group_q, bool allow_cluster, int* n_split,
+                          int* stages, int* threads, int* smem, int64_t* ctas, int* cluster, int* rows);
 size_t attn_partial_bytes();  // bytes of `partial` any launch needs
 cudaError_t launch_sparse_attn(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,
                                const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,

@@ -38,6 +38,7 @@ EXPORTED = (
     "qsa_pool_block_keys", "qsa_index_scores", "qsa_topk_blocks", "qsa_sparse_attn", "qsa_forward",
     "qsa_sparse_attn_noalloc", "qsa_sparse_attn_ex", "qsa_select_blocks",
     "qsa_cp_workspace_bytes", "qsa_cp_select_keys", "qsa_cp_merge_keys", "qsa_cp_attn_partial", "qsa_cp_combine",
+    "qsa_attn_plan",
 )
 
 CP_PART_ROW = 132  # floats per (query, head) partial of a context shard
@@ -81,6 +82,14 @@ class qsa_attn_args(ctypes.Structure):
     ]
 
 
+class qsa_attn_plan_info(ctypes.Structure):
+    _fields_ = [
+        ("n_split", ctypes.c_int32), ("n_stages", ctypes.c_int32), ("threads", ctypes.c_int32),
+        ("smem_bytes", ctypes.c_int32), ("ctas", ctypes.c_int64), ("cluster_merge", ctypes.c_int32),
+        ("rows", ctypes.c_int32),
+    ]
+
+
 _lib = None
 
 
@@ -114,6 +123,7 @@ def load(path=LIB_PATH):
     L.qsa_cp_merge_keys.argtypes = [D, I32, P, P, I32, I64, P, P, P, P, P]
     L.qsa_cp_attn_partial.argtypes = [D, P, P, P, P, P, I32, I64, P, P, P, P, SZ, P]
     L.qsa_cp_combine.argtypes = [D, I32, P, I32, P, P]
+    L.qsa_attn_plan.argtypes = [D, I32, I32, ctypes.POINTER(qsa_attn_plan_info)]
     for name in EXPORTED:
         if name not in ("qsa_workspace_bytes", "qsa_status_string", "qsa_cp_workspace_bytes"):
             getattr(L, name).restype = ctypes.c_int
@@ -222,6 +232,14 @@ def qsa_sparse_attn_ex(dims, *, q, k_cache, v_cache, q_seq, q_pos, sel_idx, sel_
     _check("qsa_sparse_attn_ex", load().qsa_sparse_attn_ex(ctypes.byref(dims), ctypes.byref(args), _ptr(workspace),
                                                            workspace.numel() * workspace.element_size(),
                                                            _stream(stream)))
+
+
+def qsa_attn_plan(dims, n_q, group_q=1):
+    """The attention launch for n_q queries in groups of group_q (host arithmetic only):
+    a dict of splits, stages, threads, shared memory, CTAs, cluster merge and rows."""
+    info = qsa_attn_plan_info()
+    _check("qsa_attn_plan", load().qsa_attn_plan(ctypes.byref(dims), n_q, group_q, ctypes.byref(info)))
+    return {name: getattr(info, name) for name, _ in qsa_attn_plan_info._fields_}
 
 
 def qsa_forward(dims, *, q, k_cache, v_cache, idx_k, pooled, q_idx, w, len_before, len_after, q_seq, q_pos,

@@ -245,6 +245,24 @@ typedef struct qsa_attn_args {
 int qsa_sparse_attn_ex(const qsa_dims* dims, const qsa_attn_args* args, void* workspace, size_t ws_bytes,
                        void* stream);
 
+/* The launch qsa_sparse_attn_ex (and the forward's attention step) makes for n_q
+ * queries in groups of group_q: host arithmetic only, no device work, usable for
+ * capacity planning.  Few (query group, KV head) pairs split each group's block list
+ * over several CTAs; at least 148 pairs take one CTA per pair.  Returns QSA_OK and
+ * fills *info, or the argument error qsa_sparse_attn_ex would return.  The cluster
+ * merge is reported as the device would run it (0 without a device). */
+typedef struct qsa_attn_plan_info {
+    int32_t n_split;        /* CTAs per (query group, KV head) */
+    int32_t n_stages;       /* K/V stages (64 tokens of K and V each) in flight per CTA */
+    int32_t threads;        /* threads per CTA */
+    int32_t smem_bytes;     /* dynamic shared memory per CTA */
+    int64_t ctas;           /* CTAs of the launch */
+    int32_t cluster_merge;  /* 1: the splits merge over distributed shared memory */
+    int32_t rows;           /* query-head rows per CTA: group_q x (n_q_heads / n_kv_heads) */
+} qsa_attn_plan_info;
+
+int qsa_attn_plan(const qsa_dims* dims, int32_t n_q, int32_t group_q, qsa_attn_plan_info* info);
+
 /* All inputs of one layer call (see the layouts above). */
 typedef struct qsa_forward_args {
     const void* q;            /* bf16 [n_q][n_q_heads][head_dim] */

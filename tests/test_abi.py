@@ -175,3 +175,36 @@ def test_workspace_grows_with_queries_and_blocks(qsa):
             assert w >= prev > 0 or prev == 0
             prev = w
         assert qsa.qsa_workspace_bytes(d, 256, 1 << 12, mode) <= qsa.qsa_workspace_bytes(d, 256, 1 << 16, mode)
+
+
+def test_attention_plans_fit_the_hardware(qsa):
+    """Every attention launch shape (host arithmetic of qsa_attn_plan, no device work):
+    shared memory within the 227 KB a CTA may use (plus its 1 KB of static alignment),
+    two CTAs per SM for the one-CTA-per-pair plan, split partials within the 148
+    slots the workspace holds, at most 6 stages, at most 32 rows per CTA."""
+    import itertools
+    max_block = 227 * 1024
+    per_sm = 228 * 1024
+    for (hq, hkv), gq, bs, n_groups in itertools.product(
+            [(8, 1), (32, 4), (16, 16), (16, 1), (32, 1), (32, 2), (4, 2), (64, 8)], [1, 2, 3, 4, 8],
+            [1, 2, 4, 8, 16], [1, 2, 3, 5, 16, 37, 64, 147, 148, 300, 4096]):
+        G = hq // hkv
+        d = qsa.make_dims(4, hq, hkv, 65536, block_size=bs)
+        n_q = n_groups * gq
+        if G * gq > 32:
+            with pytest.raises(qsa.QsaError):
+                qsa.qsa_attn_plan(d, n_q, gq)
+            continue
+        p = qsa.qsa_attn_plan(d, n_q, gq)
+        pairs = n_groups * hkv
+        assert p["rows"] == G * gq
+        assert p["threads"] == (256 if p["rows"] <= 16 else 128)
+        assert 1 <= p["n_stages"] <= 6
+        assert p["smem_bytes"] + 1024 <= max_block, p
+        assert p["ctas"] == pairs * p["n_split"]
+        if p["n_split"] > 1:
+            assert p["ctas"] <= 148, p
+        elif pairs >= 148:
+            assert 2 * (p["smem_bytes"] + 2048) <= per_sm, p
+    empty = qsa.qsa_attn_plan(qsa.make_dims(4, 32, 4, 65536), 0)
+    assert empty["ctas"] == 0
