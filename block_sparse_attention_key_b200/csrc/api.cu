@@ -88,9 +88,11 @@ WsLayout plan_workspace(const qsa_dims& d, int32_t n_q, int64_t max_blocks, int3
     L.chunk = select_chunk(max_blocks, rows);
     L.n_chunks = max_blocks > 0 ? (int)((max_blocks + L.chunk - 1) / L.chunk) : 0;
 
-    // zeroed region: attention split counters, then the select control blocks
+    // zeroed region: attention split counters, then the select control blocks.  The
+    // counters' region has one size in every layout, so calls of any shape that share
+    // a workspace find only counters there (each left at zero by its last split)
     L.attn_cnt = off;
-    L.ctrl = off + align_up((size_t)n_q * d.n_kv_heads * 4);
+    L.ctrl = off + align_up(attn_counter_bytes());
     L.ctrl_bytes = (L.ctrl - L.attn_cnt) + (size_t)rows * sizeof(TopkCtrl);
     off = L.attn_cnt + align_up(L.ctrl_bytes);
     L.cand = off;
@@ -170,8 +172,10 @@ static cudaError_t run_select(const qsa_dims& d, const void* q_idx, const float*
                            L.chunk, L.n_chunks, ctrl, (unsigned long long*)(ws + L.cand), (int32_t*)(ws + L.tmp), sel_idx, sel_cnt, true,
                            status, st, pdl);
     }
-    // prefill chunk: tensor-core scoring with streaming admission
-    e = cudaMemsetAsync(ws + L.pf_theta, 0, (size_t)(n_rows + 1) * 4, st);
+    // prefill chunk: tensor-core scoring with streaming admission.  The rows' thresholds
+    // and the fallback worklist's count start at zero; the count sits after the
+    // thresholds of the layout's n_q rows, which a mixed call's n_rows may be fewer than
+    e = cudaMemsetAsync(ws + L.pf_theta, 0, L.pf_work + 4 - L.pf_theta, st);
     if (e != cudaSuccess) return e;
     return launch_prefill_select(d, q_idx, w, pooled, q_seq, q_pos, n_rows, max_blocks, L.pf_split,
                                  (unsigned long long*)(ws + L.pf_cand), (unsigned*)(ws + L.pf_cnt),

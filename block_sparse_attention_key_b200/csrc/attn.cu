@@ -778,6 +778,12 @@ int attn_split_bound(int64_t pairs)
     return (int)(want > kDecodeMaxSplits ? kDecodeMaxSplits : want);
 }
 
+size_t attn_counter_bytes()
+{
+    // only split launches count arrivals, and they have fewer than 148 pairs
+    return (size_t)kMaxPartialSlots * 4;
+}
+
 size_t attn_partial_bytes()
 {
     // a launch splits only when (groups x KV heads) < 148, into at most

@@ -189,6 +189,7 @@ int attn_split_bound(int64_t pairs);
 bool describe_sparse_attn(const qsa_dims& d, int64_t n_groups, int group_q, bool allow_cluster, int* n_split,
                           int* stages, int* threads, int* smem, int64_t* ctas, int* cluster, int* rows);
 size_t attn_partial_bytes();  // bytes of `partial` any launch needs
+size_t attn_counter_bytes();  // bytes of `counters` any launch needs (one word per split pair)
 cudaError_t launch_sparse_attn(const qsa_dims& d, const void* q, const void* k_cache, const void* v_cache,
                                const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel_idx,
                                const int32_t* sel_cnt, const int32_t* page_table, int page_tokens, int64_t n_pages,

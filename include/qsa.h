@@ -116,7 +116,10 @@ size_t qsa_workspace_bytes(const qsa_dims* dims, int32_t n_q, int64_t max_blocks
 
 /* Zero the whole workspace (its status word and the attention's split counters,
  * which every call leaves at zero again).  Call once after allocating a workspace,
- * before its first use. */
+ * before its first use.  One workspace may then serve calls of any entry point and
+ * shape in turn (one call at a time), as long as each call's ws_bytes suffices: the
+ * counters have the same place in every call's layout, and every other region is
+ * written by the call that reads it. */
 int qsa_workspace_init(void* workspace, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, copy the device status word (QSA_DEV_* bits, 0 = clean)

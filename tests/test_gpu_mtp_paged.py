@@ -202,6 +202,77 @@ def test_bad_page_entry_is_reported_and_skipped():
     assert torch.isfinite(out.float()).all()
 
 
+def _mixed_workload(n_pf):
+    """Three decode queries of three sequences, then an n_pf-query prefill chunk of a
+    fourth sequence (16K capacity, 32 / 4 heads)."""
+    dec = [(0, 16383), (1, 12001), (2, 702)]
+    t0 = 9000
+    q_seq = [s for s, _ in dec] + [3] * n_pf
+    q_pos = [t for _, t in dec] + list(range(t0, t0 + n_pf))
+    lb = [t for _, t in dec] + [t0]
+    la = [t + 1 for _, t in dec] + [t0 + n_pf]
+    return len(dec), W.Workload("mixed", 64, "prefill", 4, 32, 4, 16384,
+                                [W.Step(lb, la, q_seq, q_pos, list(range(len(q_pos))))])
+
+
+def _forward_mixed(dw, T, m, n_dec, ws, q_idx=None):
+    """qsa_forward in QSA_MODE_MIXED over the step's first m rows."""
+    import block_sparse_attention_key_b200 as qsa
+    wl = dw.wl
+    out = torch.empty((m, wl.n_q_heads, 128), dtype=torch.bfloat16, device="cuda")
+    sel = torch.empty((m, 512), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((m,), dtype=torch.int32, device="cuda")
+    qi = T["q_idx"] if q_idx is None else q_idx
+    qsa.qsa_forward(gu.dims_of(wl), q=T["q"][:m], k_cache=dw.k_cache, v_cache=dw.v_cache, idx_k=dw.idx_k,
+                    pooled=dw.pooled, q_idx=qi[:m], w=T["w"][:m], len_before=T["len_before"],
+                    len_after=T["len_after"], q_seq=T["q_seq"][:m], q_pos=T["q_pos"][:m], n_q=m,
+                    max_new_tokens=T["max_new_tokens"], max_blocks=T["max_blocks"], mode=qsa.QSA_MODE_MIXED,
+                    out=out, workspace=ws, sel_idx=sel, sel_cnt=cnt, n_decode=n_dec)
+    return out, sel, cnt
+
+
+def test_forward_mixed_calls_with_fallback_rows_share_a_workspace():
+    """One workspace, two mixed calls.  In the first every prefill row's indexer query
+    is zero, so all its scores tie, which sends the prefill rows to the fallback select
+    (each keeps blocks 0..511); the second has fewer prefill rows and ordinary inputs
+    and must match the oracle (the fallback's worklist starts empty in every call)."""
+    import block_sparse_attention_key_b200 as qsa
+    from qsa_synth import device as sdev
+    n_dec, wl = _mixed_workload(150)
+    dw = sdev.DeviceWorkload(wl)
+    gu.pool_history(dw, 0)
+    T = dw.step_tensors(0)
+    n = T["n_q"]
+    ws = gu.new_workspace(qsa.qsa_workspace_bytes(gu.dims_of(wl), n, T["max_blocks"], qsa.QSA_MODE_MIXED))
+    wo = O.WorkloadOracle(wl)
+    q_tie = T["q_idx"].clone()
+    q_tie[n_dec:] = 0
+    _, sel, cnt = _forward_mixed(dw, T, n, n_dec, ws, q_idx=q_tie)
+    assert qsa.qsa_read_device_status(ws) == 0
+    sel, cnt = sel.cpu().numpy(), cnt.cpu().numpy()
+    for r in range(n):
+        if r < n_dec:
+            np.testing.assert_array_equal(sel[r, : cnt[r]], wo.query(0, r)[0], err_msg=f"row {r}")
+        else:
+            n_c = (wl.steps[0].q_pos[r] + 1) // 4
+            assert cnt[r] == min(512, n_c)
+            np.testing.assert_array_equal(sel[r, : cnt[r]], np.arange(cnt[r]), err_msg=f"row {r}")
+    m = n_dec + 100
+    out, sel, cnt = _forward_mixed(dw, T, m, n_dec, ws)
+    assert qsa.qsa_read_device_status(ws) == 0
+    sel, cnt = sel.cpu().numpy(), cnt.cpu().numpy()
+    rows = [0, 2, 3, 50, m - 1]
+    want = np.zeros((len(rows), 32, 128))
+    for r in range(m):
+        s_want, o_want = wo.query(0, r) if (r in rows or r % 7 == 0) else (None, None)
+        if s_want is None:
+            continue
+        np.testing.assert_array_equal(sel[r, : cnt[r]], s_want, err_msg=f"row {r}")
+        if r in rows:
+            want[rows.index(r)] = o_want
+    gu.compare_outputs(gu.bf16_to_f64(out[rows]), want)
+
+
 def test_forward_mixed_decode_and_prefill_rows():
     """A serving batch in one call: three decode queries of three sequences, then a
     150-query prefill chunk of a fourth; every row against the oracle."""
