@@ -235,7 +235,7 @@ typedef struct qsa_attn_args {
     const void* v_cache;
     const int32_t* q_seq;       /* i32 [n_q] */
     const int32_t* q_pos;       /* i32 [n_q] */
-    const int32_t* sel_idx;     /* i32 [n_q / group_q][top_k] */
+    const int32_t* sel_idx;     /* i32 [n_q / group_q][QSA_SEL_CAP] */
     const int32_t* sel_cnt;     /* i32 [n_q / group_q] */
     int32_t n_q;                /* queries */
     int32_t group_q;            /* queries per shared selection (>= 1) */
@@ -283,7 +283,7 @@ typedef struct qsa_forward_args {
     int32_t max_new_tokens;   /* host bound on len_after - len_before */
     int64_t max_blocks;       /* host bound on n_c(q_pos) over all queries */
     int32_t mode;             /* QSA_MODE_DECODE or QSA_MODE_PREFILL */
-    int32_t* sel_idx;         /* optional out i32 [n_q][top_k] (NULL: kept in workspace) */
+    int32_t* sel_idx;         /* optional out i32 [n_q][QSA_SEL_CAP] (NULL: kept in workspace) */
     int32_t* sel_cnt;         /* optional out i32 [n_q] */
     void* out;                /* bf16 [n_q][n_q_heads][head_dim] */
     /* multi-token decode (QSA_MODE_DECODE only; see qsa_sparse_attn_ex): 0 or 1 =
