@@ -181,7 +181,8 @@ def test_attention_plans_fit_the_hardware(qsa):
     """Every attention launch shape (host arithmetic of qsa_attn_plan, no device work):
     shared memory within the 227 KB a CTA may use (plus its 1 KB of static alignment),
     two CTAs per SM for the one-CTA-per-pair plan, split partials within the 148
-    slots the workspace holds, at most 6 stages, at most 32 rows per CTA."""
+    slots the workspace holds and split pairs within its 148 arrival counters, at
+    most 6 stages, at most 32 rows per CTA."""
     import itertools
     max_block = 227 * 1024
     per_sm = 228 * 1024
@@ -204,6 +205,8 @@ def test_attention_plans_fit_the_hardware(qsa):
         assert p["ctas"] == pairs * p["n_split"]
         if p["n_split"] > 1:
             assert p["ctas"] <= 148, p
+            # arrivals are counted per pair in a fixed region of 148 words
+            assert pairs < 148, p
         elif pairs >= 148:
             assert 2 * (p["smem_bytes"] + 2048) <= per_sm, p
     empty = qsa.qsa_attn_plan(qsa.make_dims(4, 32, 4, 65536), 0)
