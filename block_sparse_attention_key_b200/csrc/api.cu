@@ -37,6 +37,7 @@ int check_dims(const qsa_dims* d)
     if (d->head_dim != kHeadDim || d->n_idx_heads != kIdxHeads || d->idx_dim != kIdxDim)
         return QSA_ERR_UNSUPPORTED;
     if (d->n_q_heads / d->n_kv_heads > kMaxGroup) return QSA_ERR_UNSUPPORTED;
+    if (d->batch > 65535) return QSA_ERR_UNSUPPORTED;  // sequences index a grid dimension of the pooling launch
     return QSA_OK;
 }
 

@@ -95,7 +95,7 @@ extern "C" {
                                 chunks; one call, one attention launch over every row */
 
 typedef struct qsa_dims {
-    int32_t batch;        /* B, number of sequences (caches) */
+    int32_t batch;        /* B, number of sequences (caches): 1 .. 65535 */
     int32_t n_q_heads;    /* main attention query heads (multiple of n_kv_heads, group <= 32) */
     int32_t n_kv_heads;   /* main attention KV heads */
     int32_t head_dim;     /* must be 128 */

@@ -63,7 +63,8 @@ def test_workspace_bytes_rejects_bad_dims(qsa):
     assert ok > 0
     bad = [dict(block_size=3), dict(block_size=0), dict(block_size=32), dict(top_k=0), dict(top_k=513),
            dict(head_dim=64), dict(idx_dim=32), dict(n_idx_heads=2), dict(n_q_heads=30), dict(kv_capacity=65537),
-           dict(batch=0), dict(n_q_heads=128, n_kv_heads=2), dict(block_size=16, kv_capacity=65544)]
+           dict(batch=0), dict(batch=65536), dict(n_q_heads=128, n_kv_heads=2),
+           dict(block_size=16, kv_capacity=65544)]
     for kw in bad:
         assert qsa.qsa_workspace_bytes(_dims(qsa, **kw), 16, 16384, 0) == 0, kw
     # other micro-block sizes and budgets: per-token selection (block 1), coarser blocks, smaller k
