@@ -212,3 +212,67 @@ def test_attention_plans_fit_the_hardware(qsa):
             assert 2 * (p["smem_bytes"] + 2048) <= per_sm, p
     empty = qsa.qsa_attn_plan(qsa.make_dims(4, 32, 4, 65536), 0)
     assert empty["ctas"] == 0
+
+
+def _header_rules(d, n_q, group_q):
+    """The argument rules include/qsa.h states, restated: None when qsa_attn_plan must
+    accept (d, n_q, group_q), else the error class it must return."""
+    import math
+    invalid = (d["batch"] < 1 or d["n_q_heads"] < 1 or d["n_kv_heads"] < 1
+               or d["n_q_heads"] % d["n_kv_heads"] != 0
+               or d["block_size"] not in (1, 2, 4, 8, 16) or not 1 <= d["top_k"] <= 512
+               or d["kv_capacity"] <= 0 or d["kv_capacity"] % d["block_size"] != 0 or d["kv_capacity"] >= 2 ** 31
+               or not math.isfinite(d["softmax_scale"]))
+    if invalid:
+        return "invalid"
+    G = d["n_q_heads"] // d["n_kv_heads"]
+    if d["head_dim"] != 128 or d["n_idx_heads"] != 4 or d["idx_dim"] != 64 or G > 32 or d["batch"] > 65535:
+        return "unsupported"
+    if n_q < 0:
+        return "invalid"
+    if n_q > 65535:
+        return "unsupported"
+    if group_q < 1 or n_q % group_q != 0:
+        return "invalid"
+    if group_q * G > 32:
+        return "unsupported"
+    return None
+
+
+def test_host_checks_follow_the_header_rules(qsa):
+    """Random dims, query counts and draft-group sizes: qsa_attn_plan (host arithmetic
+    only) and qsa_workspace_bytes accept exactly what the header's rules allow and
+    return the error class they name.  Each example starts from valid dims and breaks
+    up to two fields."""
+    from hypothesis import given, settings, strategies as st
+    lib = qsa.load()
+    good = dict(batch=[1, 3, 16, 65535], heads=[(8, 1), (32, 4), (16, 16), (32, 1), (64, 2), (12, 4), (64, 8)],
+                head_dim=[128], n_idx_heads=[4], idx_dim=[64], block_size=[1, 2, 4, 8, 16], top_k=[1, 200, 512],
+                kv_capacity=[4096, 65536, 2 ** 31 - 16], softmax_scale=[0.0, 0.1])
+    bad = dict(batch=[0, -1, 65536], heads=[(30, 4), (0, 1), (4, 0), (128, 2), (66, 2)], head_dim=[64],
+               n_idx_heads=[2], idx_dim=[32], block_size=[0, 3, 32], top_k=[0, -1, 513],
+               kv_capacity=[0, 65540, 2 ** 31], softmax_scale=[float("inf"), float("nan")])
+    base_st = st.fixed_dictionaries({k: st.sampled_from(v) for k, v in good.items()})
+    breaks_st = st.lists(st.sampled_from([(k, v) for k, vs in bad.items() for v in vs]), max_size=2)
+
+    @settings(max_examples=600, deadline=None, derandomize=True)
+    @given(base_st, breaks_st, st.sampled_from([-1, 0, 1, 6, 16, 96, 65535, 65536]),
+           st.sampled_from([-1, 0, 1, 2, 3, 4, 8]))
+    def check(base, breaks, n_q, group_q):
+        d = dict(base)
+        d.update(breaks)
+        d["n_q_heads"], d["n_kv_heads"] = d.pop("heads")
+        dims = qsa.make_dims(d["batch"], d["n_q_heads"], d["n_kv_heads"], d["kv_capacity"], d["head_dim"],
+                             d["n_idx_heads"], d["idx_dim"], d["block_size"], d["top_k"], d["softmax_scale"])
+        want = _header_rules(d, n_q, group_q)
+        info = qsa.qsa_attn_plan_info()
+        rc = lib.qsa_attn_plan(ctypes.byref(dims), n_q, group_q, ctypes.byref(info))
+        expect = {None: qsa.QSA_OK, "invalid": qsa.QSA_ERR_INVALID_ARG, "unsupported": qsa.QSA_ERR_UNSUPPORTED}
+        assert rc == expect[want], (d, n_q, group_q, rc)
+        if want is None and n_q > 0:
+            assert info.ctas >= 1 and info.rows == group_q * (d["n_q_heads"] // d["n_kv_heads"])
+        # the workspace query accepts the same dims and query counts (no groups there)
+        ws_ok = _header_rules(d, n_q, 1) is None
+        assert (qsa.qsa_workspace_bytes(dims, n_q, 0, qsa.QSA_MODE_DECODE) > 0) == ws_ok, (d, n_q)
+
+    check()
